@@ -1,0 +1,51 @@
+"""The seeded input generator: determinism, block independence, dtype exactness."""
+import numpy as np
+
+import workloads
+
+
+def test_blocks_are_deterministic_and_independent():
+    wl = workloads.get("tiny").with_(B=2, H_q=2, H_kv=2, S=64)
+    a = workloads.keys_block(wl, 1, 1)
+    b = workloads.keys_block(wl, 1, 1)
+    np.testing.assert_array_equal(a, b)
+    assert not np.array_equal(a, workloads.keys_block(wl, 0, 1))
+    full = workloads.generate(wl, threads=2)
+    np.testing.assert_array_equal(full["K"][1, 1], a)
+    np.testing.assert_array_equal(full["V"][0, 1], workloads.values_block(wl, 0, 1))
+    np.testing.assert_array_equal(full["q"][1, 0], workloads.query_vec(wl, 1, 0))
+    assert full["K_cal"].shape == (wl.n_cal, 2, wl.D)
+
+
+def test_bf16_values_are_exact():
+    wl = workloads.get("llama2-7b").with_(S=128, H_q=2, H_kv=2)
+    K = workloads.keys_block(wl, 0, 0)
+    bits = workloads.bf16_bits(K)
+    back = (bits.astype(np.uint32) << 16).view(np.float32)
+    np.testing.assert_array_equal(back, K)
+
+
+def test_rotation_is_orthogonal():
+    wl = workloads.get("llama3-8b-gqa")
+    R = workloads.rotation(wl, 3)
+    np.testing.assert_allclose(R.T @ R, np.eye(wl.D), atol=1e-12)
+
+
+def test_gqa_queries_use_their_kv_head_basis():
+    wl = workloads.get("llama3-8b-gqa")
+    # the query of head 5 lives in KV head 1's subspace: its energy sits in the
+    # leading columns of that head's R, not of another head's
+    q = workloads.query_vec(wl, 0, 5).astype(np.float64)
+    e_own = np.sum((q @ workloads.rotation(wl, 1))[:8] ** 2)
+    e_other = np.sum((q @ workloads.rotation(wl, 2))[:8] ** 2)
+    assert e_own > 4 * e_other
+
+
+def test_sweep_has_54_points_and_sample_rows():
+    pts = workloads.sweep_points()
+    assert len(pts) == 54
+    assert all(p.k * 8 == p.S or p.k * 4 == p.S for p in pts)
+    wl = workloads.get("llama2-13b")
+    rows = workloads.sample_rows(wl, 16)
+    assert len(rows) == 16 and rows[0] == (0, 0) and rows[-1] == (wl.B - 1, wl.H_q - 1)
+    assert len(set(rows)) == 16
