@@ -1,0 +1,489 @@
+#!/usr/bin/env python
+"""Loki decode-attention benchmark on B200.
+
+One step = one Loki decode layer-step (project q, low-dim score scan, top-k,
+sparse attention over the selected tokens, combine) over the Llama2-13B-shaped
+batched decode workload (B = 16, H = 40, D = 128, S = 4096, d = 32, k = 512,
+bf16), with the KV-cache resident in HBM. Inputs are seeded synthetic
+low-rank keys; the PCA basis is calibrated and the cache is filled through the
+library itself (loki_calibrate_pca, loki_append_keys) before timing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0. `value` is microseconds per layer-step for the
+whole job (max-over-ranks device time / (K * N)); lower is better. L2 is
+flushed (a 256 MiB write) before every timed step; flush time is excluded.
+Multi-GPU runs (torchrun) are weak-scaled replicas: the path has no exchange
+step, so ranks share nothing but the final max-reduction of their timings.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (this tier has no runnable upstream code).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Loki decode-attn µs/layer-step, HBM GB/s (% roofline), speedup vs dense"
+UNIT = "us/layer-step"
+FALLBACK_HBM_GBS = 6650.0
+LAUNCHES_PER_DECODE = 5  # project, score, top-k, sparse attention, combine
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2-13b")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every 5 ms."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, torch_device_index: int):
+        self.samples, self.reasons = [], set()
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hh)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hh
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.nvml, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": getattr(self, "err", "no samples")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def traffic_from_profiles(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if its source hash is current."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.e+]+)", txt)
+    m_h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_f = re.search(r"source_file:\s*(\S+)", txt)
+    if not (m_t and m_h and m_f):
+        return None
+    src = os.path.join(ROOT, m_f.group(1))
+    if not os.path.exists(src):
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != m_h.group(1):
+        return None
+    return float(m_t.group(1))
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (rank 0 only)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rows(wl, n_rows, seed=11):
+    """Host inputs of a seeded sample of (b, h_q) rows: q, K~ (oracle-rotated), V, P."""
+    import numpy as np
+
+    import oracle
+    import workloads
+    rows = workloads.sample_rows(wl, n_rows, seed)
+    cache = {}
+    out = []
+    for b, h in rows:
+        hk = h // wl.G
+        if ("P", hk) not in cache:
+            R = workloads.rotation(wl, hk)
+            P, _ = oracle.calibrate_pca(workloads.calibration_keys(wl, hk, R))
+            cache[("P", hk)] = (R, P.astype(np.float32).astype(np.float64))
+        R, P = cache[("P", hk)]
+        if (b, hk) not in cache:
+            K = workloads.keys_block(wl, b, hk, R)
+            cache[(b, hk)] = (oracle.rotate_keys(K, P, wl.dtype),
+                              workloads.values_block(wl, b, hk).astype(np.float64))
+        Kt, V = cache[(b, hk)]
+        out.append((workloads.query_vec(wl, b, h, R).astype(np.float64), Kt, V, P))
+    return out
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_oracle_time(wl, seconds: float, rows_per_step: int = 0):
+    """Time oracle.loki_decode_row over sampled rows; returns (us per layer-step, info)."""
+    import oracle
+    sample = oracle_sample_rows(wl, 8)
+    per_row = []
+    t_end = time.perf_counter() + seconds
+    i = 0
+    while (time.perf_counter() < t_end or len(per_row) < 4) and len(per_row) < 100000:
+        q, Kt, V, P = sample[i % len(sample)]
+        t0 = time.perf_counter()
+        oracle.loki_decode_row(q, Kt, V, P, wl.d, wl.k, wl.scale)
+        per_row.append(time.perf_counter() - t0)
+        i += 1
+    mean_row = sum(per_row) / len(per_row)
+    rows = wl.B * wl.H_q
+    return mean_row * rows * 1e6, {
+        "rows_timed": len(per_row), "distinct_rows": len(sample),
+        "cores": blas_threads(), "host_cores": host_cores()}
+
+
+# ---------------------------------------------------------------------------
+# GPU benchmark
+# ---------------------------------------------------------------------------
+
+def build_gpu_inputs(wl, dev, rank):
+    """Seeded inputs on the device; P and the rotated cache come from the library."""
+    import numpy as np
+    import torch
+
+    import sparse_attention_decode_loki_b200 as loki
+    import workloads
+    wl_r = wl.with_(seed=wl.seed + 1_000_000 * rank) if rank else wl
+    g = workloads.generate(wl_r)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    K_cal = torch.from_numpy(g["K_cal"]).to(dev).to(dt)
+    P, eig = loki.loki_calibrate_pca(K_cal)
+    S_max = wl.S
+    Kt = torch.empty((wl.B, wl.H_kv, S_max, wl.D), dtype=dt, device=dev)
+    V = torch.empty_like(Kt)
+    K_raw = torch.from_numpy(g.pop("K")).to(dev).to(dt)
+    V_raw = torch.from_numpy(g.pop("V")).to(dev).to(dt)
+    loki.loki_append_keys(K_raw, V_raw, P, Kt, V, 0)
+    # the new token of the timed append (one per sequence and KV head)
+    K_new = K_raw[:, :, -1:].contiguous()
+    V_new = V_raw[:, :, -1:].contiguous()
+    del K_raw, V_raw
+    q = torch.from_numpy(g["q"]).to(dev).to(dt)
+    torch.cuda.synchronize()
+    return {"q": q, "Kt": Kt, "V": V, "P": P, "eig": eig, "K_new": K_new, "V_new": V_new,
+            "q_host": g["q"]}
+
+
+def run_ours(args):
+    import torch
+
+    import sparse_attention_decode_loki_b200 as loki
+    import workloads
+
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    wl = workloads.get(args.workload)
+    inp = build_gpu_inputs(wl, dev, rank)
+    q, Kt, V, P = inp["q"], inp["Kt"], inp["V"], inp["P"]
+    B, H_q, H_kv, S, D, d, k = wl.B, wl.H_q, wl.H_kv, wl.S, wl.D, wl.d, wl.k
+    e = wl.elem_bytes
+    out = torch.empty_like(q)
+    idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    ws = torch.empty(loki.loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def decode():
+        loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
+                                   workspace=ws)
+
+    def timed(fn, n, warm):
+        for _ in range(warm):
+            flush.zero_()
+            fn()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            starts[i].record(stream)
+            fn()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        return [s.elapsed_time(t) for s, t in zip(starts, ends)]
+
+    # ---- the timed region: exactly K decode steps --------------------------------
+    for _ in range(args.warmup):
+        flush.zero_()
+        decode()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms = timed(decode, args.steps, 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    us_per_step_rank = total_ms * 1e3 / args.steps
+    value = us_per_step_rank / world
+
+    # ---- per-kernel breakdown through the step entry points ----------------------
+    q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
+    scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
+    sp_ws = torch.empty(loki.loki_sparse_attention_workspace_size(B, H_q, k, D), dtype=torch.uint8,
+                        device=dev)
+    nb = max(50, min(args.steps, 400))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nb)]
+    for i in range(nb + 10):
+        flush.zero_()
+        ev = evs[i - 10] if i >= 10 else None
+        if ev: ev[0].record(stream)
+        loki.loki_project_query(q, P, q_rot)
+        if ev: ev[1].record(stream)
+        loki.loki_score_lowdim(q_rot, Kt, S, d, scores)
+        if ev: ev[2].record(stream)
+        loki.loki_topk(scores, k, idx)
+        if ev: ev[3].record(stream)
+        loki.loki_sparse_attention(q_rot, Kt, V, idx, S, wl.scale, out, sp_ws)
+        if ev: ev[4].record(stream)
+    torch.cuda.synchronize()
+    names = ["project_query", "score_lowdim", "topk", "sparse_attention+combine"]
+    kern_us = {n: statistics.mean(e_[j].elapsed_time(e_[j + 1]) for e_ in evs) * 1e3
+               for j, n in enumerate(names)}
+
+    # ---- dense baseline on the same cache (q~ rounded to the cache dtype) ------
+    q_rot_dt = loki.loki_project_query(q, P).to(q.dtype)
+    dws = torch.empty(loki.dense_decode_workspace_size(B, H_q, H_kv, S, D), dtype=torch.uint8,
+                      device=dev)
+    dout = torch.empty_like(q)
+    dense_ms = timed(lambda: loki.dense_decode_attention(q_rot_dt, Kt, V, S, wl.scale, dout, dws),
+                     nb, 10)
+    dense_us = statistics.mean(dense_ms) * 1e3
+
+    # ---- append of one new token per (sequence, KV head) -------------------------
+    Kt_app = torch.empty((B, H_kv, 8, D), dtype=q.dtype, device=dev)
+    V_app = torch.empty_like(Kt_app)
+    app_ms = timed(lambda: loki.loki_append_keys(inp["K_new"], inp["V_new"], P, Kt_app, V_app, 0),
+                   nb, 10)
+    append_us = statistics.mean(app_ms) * 1e3
+
+    # ---- end to end through the public API with host buffers ---------------------
+    q_pin = torch.from_numpy(inp["q_host"]).to(q.dtype).pin_memory()
+    out_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    idx_pin = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(q_pin, non_blocking=True)
+        decode()
+        out_pin.copy_(out, non_blocking=True)
+        idx_pin.copy_(idx, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, max(50, min(args.steps, 1000)), 5)
+    e2e_us = statistics.mean(e2e_ms) * 1e3
+    if world > 1:
+        t = torch.tensor([e2e_us], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_us = float(t.item())
+    h2d = q_pin.numel() * q_pin.element_size()
+    d2h = out_pin.numel() * out_pin.element_size() + idx_pin.numel() * idx_pin.element_size()
+
+    # ---- roofline of the dominant kernel ------------------------------------------
+    peak, peak_kind = load_peaks()
+    alg = {
+        "score_lowdim": e * B * H_kv * S * d,
+        "sparse_attention+combine": e * B * H_q * 2 * k * D,
+    }
+    dom = max(alg, key=lambda n: kern_us[n])
+    achieved = alg[dom] / (kern_us[dom] * 1e-6) / 1e9
+    step_bytes = wl.loki_bytes()
+    step_us = us_per_step_rank
+    prof_name = {"score_lowdim": "score_lowdim", "sparse_attention+combine": "sparse_attn"}[dom]
+    traffic = traffic_from_profiles(prof_name, wl.name)
+
+    res = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(us_per_step_rank / 1e3, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded low-rank keys, N(0,1) values; PCA and cache built by the library)",
+        "config": {"workload": wl.name, "B": B, "H_q": H_q, "H_kv": H_kv, "D": D, "S": S,
+                   "d": d, "k": k, "cache_dtype": wl.dtype,
+                   "l2": "flushed (256 MiB write) before every timed step, flush excluded",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "tokens_per_s": round(B * world * 1e6 / us_per_step_rank, 1),
+        "hbm_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
+        "hbm_frac_of_" + peak_kind: round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 4),
+        "dense_us": round(dense_us, 3),
+        "speedup_vs_dense": round(dense_us / step_us, 3),
+        "append_us": round(append_us, 3),
+        "kernels_us": {n_: round(v_, 3) for n_, v_ in kern_us.items()},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes": alg[dom]},
+        "e2e": {"value": round(e2e_us / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": LAUNCHES_PER_DECODE * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu_us, info = cpu_oracle_time(wl, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": round(cpu_us, 1), "unit": UNIT, "cores": info["cores"],
+                               "kind": "oracle",
+                               "sample": f"{info['rows_timed']} timed (batch, head) rows drawn "
+                                         f"from {info['distinct_rows']} seeded rows of "
+                                         f"{wl.name}, scaled by B*H_q = {B * H_q}",
+                               "host_cores": info["host_cores"]}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import workloads
+    wl = workloads.get(args.workload)
+    rows_per_step = 4
+    import oracle
+    sample = oracle_sample_rows(wl, 8)
+
+    def step(i):
+        for j in range(rows_per_step):
+            q, Kt, V, P = sample[(i * rows_per_step + j) % len(sample)]
+            oracle.loki_decode_row(q, Kt, V, P, wl.d, wl.k, wl.scale)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    per_row = dt / (args.steps * rows_per_step)
+    us = per_row * wl.B * wl.H_q * 1e6
+    sample_txt = (f"{rows_per_step} (batch, head) rows per step from 8 seeded rows of {wl.name}, "
+                  f"scaled by B*H_q = {wl.B * wl.H_q}")
+    res = {
+        "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded low-rank keys)", "impl": "reference",
+        "config": {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D,
+                   "S": wl.S, "d": wl.d, "k": wl.k, "cache_dtype": wl.dtype},
+        "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle", "sample": sample_txt},
+        "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+/*
+ * loki.h -- C ABI of the B200 (sm_100a) implementation of Loki decode-time
+ * sparse attention ("Loki: Low-Rank Keys for Efficient Sparse Attention").
+ *
+ * What the method computes (NeurIPS 2024 poster page of the paper, TL;DR and
+ * "Visual Insights" Figure 1 caption; briefgpt.xyz abstract page):
+ *   offline : a PCA basis P of each KV head's keys, from calibration keys;
+ *   append  : every key enters the KV-cache rotated, K~ = K P;
+ *   decode  : per (batch, query head), q~ = q P; approximate scores on the
+ *             first d principal components, s_j = q~[:d] . K~_j[:d]; keep the
+ *             k tokens with the largest s_j; exact softmax attention over
+ *             those k tokens with their full D-dimensional rotated keys
+ *             (q~ . K~_j = q . K_j because P is orthonormal) and values.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller. The
+ *     library never allocates, frees or synchronises; work is enqueued on
+ *     `stream`, a cudaStream_t passed as an opaque pointer (NULL = the legacy
+ *     default stream). Calls are asynchronous: device-side failures surface
+ *     at the caller's next synchronisation.
+ *   - Layouts are dense row-major with the last dimension contiguous:
+ *       q, out            [B, H_q, D]
+ *       K~ cache, V cache [B, H_kv, S_max, D]  (rows [0, S) valid)
+ *       P                 [H_kv, D, D] fp32, P[h][i][c] = entry i of
+ *                         principal component c (eigenvalue-descending)
+ *       selected_idx      [B, H_q, k] int32, ascending token index
+ *     Query head h reads KV head h / (H_q / H_kv) (grouped-query attention).
+ *   - dt is the element type of q, caches, new keys/values and out.
+ *   - Device pointers must be 16-byte aligned; workspaces 256-byte aligned.
+ *   - Arguments are checked on the host before anything is enqueued; on any
+ *     error nothing is launched and a loki_status other than LOKI_OK is
+ *     returned. loki_last_error() then describes the failing argument.
+ *   - D must be 128 (other head sizes return LOKI_ERR_UNSUPPORTED) and
+ *     H_q / H_kv must be at most 8.
+ *   - Entry points are thread-safe; calls on one stream are ordered.
+ */
+#ifndef LOKI_H
+#define LOKI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LOKI_API __attribute__((visibility("default")))
+#else
+#define LOKI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum loki_status {
+    LOKI_OK = 0,
+    LOKI_ERR_INVALID_ARG = 1,         /* null pointer, bad size, misaligned pointer */
+    LOKI_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. D != 128) */
+    LOKI_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size() figure */
+    LOKI_ERR_CUDA = 4                 /* a CUDA runtime call or launch failed */
+} loki_status;
+
+typedef enum loki_dtype {
+    LOKI_DTYPE_F32 = 0,
+    LOKI_DTYPE_BF16 = 1
+} loki_dtype;
+
+/* Text for a status code (static storage). */
+LOKI_API const char* loki_status_string(loki_status st);
+
+/* Description of the last failure on the calling thread ("" if none). */
+LOKI_API const char* loki_last_error(void);
+
+/* ------------------------------------------------------------------------ */
+/* Offline calibration                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace loki_calibrate_pca needs. */
+LOKI_API size_t loki_calibrate_workspace_size(int64_t N, int H_kv, int D);
+
+/*
+ * PCA of calibration keys, one basis per KV head. Poster page, "Visual
+ * Insights" Figure 1 caption (offline PCA on calibration keys) and the
+ * study.space summary (PCA reduces the key dimensionality).
+ *   keys    [N, H_kv, D] of type dt, N >= 2
+ *   P       out, [H_kv, D, D] fp32; column c = unit eigenvector of the
+ *           centred covariance (divisor N - 1) with the c-th largest
+ *           eigenvalue, sign chosen so its largest-magnitude entry (lowest
+ *           index on a tie) is positive
+ *   eigvals out, [H_kv, D] fp32 descending, or NULL
+ * Covariance in fp64, eigen-decomposition by cyclic Jacobi in fp64.
+ */
+LOKI_API loki_status loki_calibrate_pca(const void* keys, loki_dtype dt, int64_t N, int H_kv, int D,
+                               float* P, float* eigvals, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* KV-cache append                                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Append T new tokens per (batch, KV head): K~ = K_new P (fp32 accumulate,
+ * rounded to dt, nearest-even) into K~ cache rows [pos, pos + T); V_new is
+ * copied unchanged into the same rows of the V cache. The poster page's
+ * "Loki's Computational Cost" section names this append as a step of every
+ * decode iteration.
+ *   K_new, V_new [B, H_kv, T, D] of type dt;  P [H_kv, D, D] fp32
+ *   requires 0 <= pos and pos + T <= S_max
+ */
+LOKI_API loki_status loki_append_keys(const void* K_new, const void* V_new, const float* P,
+                             void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
+                             int64_t S_max, int64_t pos, loki_dtype dt, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention (the per-step hot path)                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace loki_decode_attention needs (q~, scores, partials). */
+LOKI_API size_t loki_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, int D, int d, int64_t k);
+
+/*
+ * One Loki decode step over a cache holding S valid tokens (poster TL;DR and
+ * Figure 1 caption; briefgpt.xyz abstract page).
+ *   q [B, H_q, D] (dt); Kt_cache, V_cache [B, H_kv, S_max, D] (dt); P fp32
+ *   1 <= d <= D, 1 <= k <= S <= S_max, S < 2^31
+ *   scale   softmax scale of the final scores; <= 0 selects 1/sqrt(D)
+ *   out     [B, H_q, D] (dt): softmax over the k selected tokens only
+ *   selected_idx [B, H_q, k] int32: the k tokens with the largest
+ *           low-dimensional score, ties to the lower index, ascending
+ * Arithmetic: fp32 (q~, scores, softmax, accumulation) on dt inputs.
+ */
+LOKI_API loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
+                                  const float* P, int B, int H_q, int H_kv, int64_t S,
+                                  int64_t S_max, int D, int d, int64_t k, float scale,
+                                  loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* Steps of loki_decode_attention, callable one by one ------------------- */
+
+/* q_rot [B, H_q, D] fp32 = q P (query rotated into its KV head's basis). */
+LOKI_API loki_status loki_project_query(const void* q, const float* P, int B, int H_q, int H_kv, int D,
+                               loki_dtype dt, float* q_rot, void* stream);
+
+/*
+ * scores [B, H_q, S] fp32: s_j = sum_{i<d} q_rot[i] K~_j[i] for j < S. Only
+ * the first d columns of each cached key are read; each KV head's rows are
+ * read once for all of its query heads.
+ */
+LOKI_API loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, int H_q, int H_kv,
+                              int64_t S, int64_t S_max, int D, int d, loki_dtype dt,
+                              float* scores, void* stream);
+
+/* Bytes of workspace loki_topk needs (currently 0; reserved). */
+LOKI_API size_t loki_topk_workspace_size(int64_t rows, int64_t S, int64_t k);
+
+/*
+ * Per row of `scores` [rows, S] fp32: the k indices of the largest values,
+ * ties to the lower index, written ascending to selected_idx [rows, k].
+ * -0.0 equals +0.0; NaN ranks below every number. 1 <= k <= S.
+ */
+LOKI_API loki_status loki_topk(const float* scores, int64_t rows, int64_t S, int64_t k,
+                      int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace loki_sparse_attention needs (split-k partials). */
+LOKI_API size_t loki_sparse_attention_workspace_size(int B, int H_q, int64_t k, int D);
+
+/*
+ * Exact attention over the selected tokens: a_j = scale q_rot . K~_j over all
+ * D dimensions for j in selected_idx[b, h, :], softmax over those k, out =
+ * sum p_j V_j. Indices outside [0, S) are skipped (they contribute nothing);
+ * a row whose indices are all out of range yields zeros.
+ */
+LOKI_API loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, const void* V_cache,
+                                  const int32_t* selected_idx, int B, int H_q, int H_kv,
+                                  int64_t S, int64_t S_max, int D, int64_t k, float scale,
+                                  loki_dtype dt, void* out, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Dense baseline                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace dense_decode_attention needs (split-S partials). */
+LOKI_API size_t dense_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, int D);
+
+/*
+ * Full decode attention over all S cached tokens, the baseline Loki is
+ * compared with (poster page, "More on tables": full attention rows;
+ * per-layer attention time figure under "More on figures"). q and K may be
+ * both rotated or both unrotated: the scores are the same.
+ *   q [B, H_q, D]; K_cache, V_cache [B, H_kv, S_max, D]; out [B, H_q, D]
+ */
+LOKI_API loki_status dense_decode_attention(const void* q, const void* K_cache, const void* V_cache,
+                                   int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D,
+                                   float scale, loki_dtype dt, void* out, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOKI_H */

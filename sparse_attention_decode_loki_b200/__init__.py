@@ -1,0 +1,243 @@
+"""Loki decode-time sparse attention on B200 (sm_100a): Python binding.
+
+Every function here only marshals torch tensors into the C ABI of libloki.so
+(include/loki.h) and allocates outputs and workspaces the caller did not pass;
+all arithmetic runs in the library's CUDA kernels on the tensors' device, on
+the current torch stream. Names match the C entry points.
+
+Loki ("Loki: Low-Rank Keys for Efficient Sparse Attention"; NeurIPS 2024
+poster page, TL;DR and "Visual Insights" Figure 1 caption): keys are cached
+rotated by a per-head PCA basis P; at each decode step the query is rotated,
+tokens are ranked by their score on the first d principal components, the
+top k are kept, and exact softmax attention runs over those k tokens only.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from ._lib import DTYPE_BF16, DTYPE_F32, LIB_PATH, LokiError, check, lib  # noqa: F401
+
+__all__ = [
+    "LokiError", "LIB_PATH",
+    "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
+    "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
+    "loki_decode_workspace_size", "dense_decode_workspace_size",
+    "loki_sparse_attention_workspace_size", "loki_calibrate_workspace_size",
+    "loki_topk_workspace_size",
+]
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: use torch.float32 or torch.bfloat16")
+
+
+def _cuda(*ts: torch.Tensor) -> torch.device:
+    dev = ts[0].device
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if t.device != dev:
+            raise ValueError("all tensors must be on the same device")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+    return dev
+
+
+def _stream(dev: torch.device) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _ws(nbytes: int, dev: torch.device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is None:
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    return ws
+
+
+def _ws_bytes(ws: torch.Tensor) -> int:
+    return ws.numel() * ws.element_size()
+
+
+# ---------------------------------------------------------------------------
+# workspace sizes
+# ---------------------------------------------------------------------------
+
+def loki_decode_workspace_size(B: int, H_q: int, H_kv: int, S: int, D: int, d: int, k: int) -> int:
+    return int(lib.loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k))
+
+
+def dense_decode_workspace_size(B: int, H_q: int, H_kv: int, S: int, D: int) -> int:
+    return int(lib.dense_decode_workspace_size(B, H_q, H_kv, S, D))
+
+
+def loki_sparse_attention_workspace_size(B: int, H_q: int, k: int, D: int) -> int:
+    return int(lib.loki_sparse_attention_workspace_size(B, H_q, k, D))
+
+
+def loki_calibrate_workspace_size(N: int, H_kv: int, D: int) -> int:
+    return int(lib.loki_calibrate_workspace_size(N, H_kv, D))
+
+
+def loki_topk_workspace_size(rows: int, S: int, k: int) -> int:
+    return int(lib.loki_topk_workspace_size(rows, S, k))
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def loki_calibrate_pca(keys: torch.Tensor, P: Optional[torch.Tensor] = None,
+                       eigvals: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """keys [N, H_kv, D] -> (P [H_kv, D, D] fp32, eigvals [H_kv, D] fp32)."""
+    dev = _cuda(keys)
+    N, H_kv, D = keys.shape
+    if P is None:
+        P = torch.empty((H_kv, D, D), dtype=torch.float32, device=dev)
+    if eigvals is None:
+        eigvals = torch.empty((H_kv, D), dtype=torch.float32, device=dev)
+    _cuda(keys, P, eigvals)
+    ws = _ws(loki_calibrate_workspace_size(N, H_kv, D), dev, workspace)
+    check(lib.loki_calibrate_pca(keys.data_ptr(), _dt(keys), N, H_kv, D, P.data_ptr(),
+                                 eigvals.data_ptr(), ws.data_ptr(), _ws_bytes(ws), _stream(dev)),
+          "loki_calibrate_pca")
+    return P, eigvals
+
+
+def loki_append_keys(K_new: torch.Tensor, V_new: torch.Tensor, P: torch.Tensor,
+                     Kt_cache: torch.Tensor, V_cache: torch.Tensor, pos: int) -> None:
+    """Rotate K_new [B, H_kv, T, D] by P and write it, with V_new, into cache rows [pos, pos+T)."""
+    dev = _cuda(K_new, V_new, P, Kt_cache, V_cache)
+    B, H_kv, T, D = K_new.shape
+    S_max = Kt_cache.shape[2]
+    if V_new.shape != K_new.shape or Kt_cache.shape != V_cache.shape:
+        raise ValueError("shape mismatch")
+    if Kt_cache.shape[:2] != (B, H_kv) or Kt_cache.shape[3] != D:
+        raise ValueError("cache shape does not match K_new")
+    for t in (V_new, Kt_cache, V_cache):
+        if t.dtype != K_new.dtype:
+            raise TypeError("K_new, V_new and the caches must share a dtype")
+    if P.dtype != torch.float32 or tuple(P.shape) != (H_kv, D, D):
+        raise ValueError("P must be float32 [H_kv, D, D]")
+    check(lib.loki_append_keys(K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+                               Kt_cache.data_ptr(), V_cache.data_ptr(), B, H_kv, T, D, S_max, pos,
+                               _dt(K_new), _stream(dev)), "loki_append_keys")
+
+
+def _check_decode(q, Kt, V, P=None):
+    dev = _cuda(q, Kt, V, *(() if P is None else (P,)))
+    B, H_q, D = q.shape
+    Bk, H_kv, S_max, Dk = Kt.shape
+    if Bk != B or Dk != D or V.shape != Kt.shape:
+        raise ValueError("q [B, H_q, D] and caches [B, H_kv, S_max, D] disagree")
+    if Kt.dtype != q.dtype or V.dtype != q.dtype:
+        raise TypeError("q and the caches must share a dtype")
+    if P is not None and (P.dtype != torch.float32 or tuple(P.shape) != (H_kv, D, D)):
+        raise ValueError("P must be float32 [H_kv, D, D]")
+    return dev, B, H_q, H_kv, S_max, D
+
+
+def loki_decode_attention(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,
+                          P: torch.Tensor, S: int, d: int, k: int, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None,
+                          selected_idx: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One Loki decode step. Returns (out [B, H_q, D], selected_idx [B, H_q, k] int32)."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q, Kt_cache, V_cache, P)
+    if out is None:
+        out = torch.empty_like(q)
+    if selected_idx is None:
+        selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    _cuda(q, out, selected_idx)
+    ws = _ws(loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k), dev, workspace)
+    check(lib.loki_decode_attention(q.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
+                                    P.data_ptr(), B, H_q, H_kv, S, S_max, D, d, k, float(scale),
+                                    _dt(q), out.data_ptr(), selected_idx.data_ptr(), ws.data_ptr(),
+                                    _ws_bytes(ws), _stream(dev)), "loki_decode_attention")
+    return out, selected_idx
+
+
+def loki_project_query(q: torch.Tensor, P: torch.Tensor,
+                       q_rot: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """q [B, H_q, D] -> q~ = q P, fp32 [B, H_q, D]."""
+    dev = _cuda(q, P)
+    B, H_q, D = q.shape
+    H_kv = P.shape[0]
+    if q_rot is None:
+        q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
+    check(lib.loki_project_query(q.data_ptr(), P.data_ptr(), B, H_q, H_kv, D, _dt(q),
+                                 q_rot.data_ptr(), _stream(dev)), "loki_project_query")
+    return q_rot
+
+
+def loki_score_lowdim(q_rot: torch.Tensor, Kt_cache: torch.Tensor, S: int, d: int,
+                      scores: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fp32 scores [B, H_q, S] on the first d rotated dimensions."""
+    dev = _cuda(q_rot, Kt_cache)
+    B, H_q, D = q_rot.shape
+    _, H_kv, S_max, _ = Kt_cache.shape
+    if q_rot.dtype != torch.float32:
+        raise TypeError("q_rot must be float32")
+    if scores is None:
+        scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
+    check(lib.loki_score_lowdim(q_rot.data_ptr(), Kt_cache.data_ptr(), B, H_q, H_kv, S, S_max, D,
+                                d, _dt(Kt_cache), scores.data_ptr(), _stream(dev)),
+          "loki_score_lowdim")
+    return scores
+
+
+def loki_topk(scores: torch.Tensor, k: int, selected_idx: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per row of scores [..., S] fp32: k indices of the largest values (ties: lower index), ascending."""
+    dev = _cuda(scores)
+    if scores.dtype != torch.float32:
+        raise TypeError("scores must be float32")
+    S = scores.shape[-1]
+    rows = scores.numel() // S
+    if selected_idx is None:
+        selected_idx = torch.empty((*scores.shape[:-1], k), dtype=torch.int32, device=dev)
+    ws = _ws(loki_topk_workspace_size(rows, S, k), dev, None)
+    check(lib.loki_topk(scores.data_ptr(), rows, S, k, selected_idx.data_ptr(), ws.data_ptr(),
+                        _ws_bytes(ws), _stream(dev)), "loki_topk")
+    return selected_idx
+
+
+def loki_sparse_attention(q_rot: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,
+                          selected_idx: torch.Tensor, S: int, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Exact attention of q~ over the selected tokens; out has the caches' dtype."""
+    dev = _cuda(q_rot, Kt_cache, V_cache, selected_idx)
+    B, H_q, D = q_rot.shape
+    _, H_kv, S_max, _ = Kt_cache.shape
+    k = selected_idx.shape[-1]
+    if selected_idx.dtype != torch.int32:
+        raise TypeError("selected_idx must be int32")
+    if out is None:
+        out = torch.empty((B, H_q, D), dtype=Kt_cache.dtype, device=dev)
+    ws = _ws(loki_sparse_attention_workspace_size(B, H_q, k, D), dev, workspace)
+    check(lib.loki_sparse_attention(q_rot.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
+                                    selected_idx.data_ptr(), B, H_q, H_kv, S, S_max, D, k,
+                                    float(scale), _dt(Kt_cache), out.data_ptr(), ws.data_ptr(),
+                                    _ws_bytes(ws), _stream(dev)), "loki_sparse_attention")
+    return out
+
+
+def dense_decode_attention(q: torch.Tensor, K_cache: torch.Tensor, V_cache: torch.Tensor, S: int,
+                           scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Full decode attention over all S cached tokens."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q, K_cache, V_cache)
+    if out is None:
+        out = torch.empty_like(q)
+    ws = _ws(dense_decode_workspace_size(B, H_q, H_kv, S, D), dev, workspace)
+    check(lib.dense_decode_attention(q.data_ptr(), K_cache.data_ptr(), V_cache.data_ptr(), B, H_q,
+                                     H_kv, S, S_max, D, float(scale), _dt(q), out.data_ptr(),
+                                     ws.data_ptr(), _ws_bytes(ws), _stream(dev)),
+          "dense_decode_attention")
+    return out

@@ -1,0 +1,388 @@
+// C ABI of the Loki library (declared in include/loki.h): argument checks,
+// workspace carving and the launch sequence of each entry point. Every check
+// runs on the host before anything is enqueued, so a rejected call launches
+// nothing and touches no device memory.
+#include <math.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/loki.h"
+#include "launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+loki_status fail(loki_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+loki_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(LOKI_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxGroup = 8;
+constexpr int64_t kMaxS = 0x7fffffff;
+
+#define LOKI_REQUIRE(cond, st, ...) \
+    do {                            \
+        if (!(cond)) return fail(st, __VA_ARGS__); \
+    } while (0)
+
+loki_status check_dtype(loki_dtype dt) {
+    LOKI_REQUIRE(dt == LOKI_DTYPE_F32 || dt == LOKI_DTYPE_BF16, LOKI_ERR_INVALID_ARG,
+                 "dt must be LOKI_DTYPE_F32 or LOKI_DTYPE_BF16 (got %d)", (int)dt);
+    return LOKI_OK;
+}
+
+loki_status check_heads(int B, int H_q, int H_kv, int D) {
+    LOKI_REQUIRE(B >= 1 && B <= 65535, LOKI_ERR_INVALID_ARG, "B must be in [1, 65535] (got %d)", B);
+    LOKI_REQUIRE(H_q >= 1 && H_kv >= 1, LOKI_ERR_INVALID_ARG, "H_q and H_kv must be >= 1");
+    LOKI_REQUIRE(H_q % H_kv == 0, LOKI_ERR_INVALID_ARG, "H_q (%d) must be a multiple of H_kv (%d)",
+                 H_q, H_kv);
+    LOKI_REQUIRE(H_q / H_kv <= kMaxGroup, LOKI_ERR_UNSUPPORTED,
+                 "H_q / H_kv = %d exceeds the supported group size %d", H_q / H_kv, kMaxGroup);
+    LOKI_REQUIRE(D >= 1, LOKI_ERR_INVALID_ARG, "D must be >= 1");
+    LOKI_REQUIRE(D == 128, LOKI_ERR_UNSUPPORTED, "D = %d: only D = 128 is implemented", D);
+    LOKI_REQUIRE((int64_t)B * H_q <= 0x7fffffff, LOKI_ERR_INVALID_ARG, "B * H_q too large");
+    return LOKI_OK;
+}
+
+loki_status check_seq(int64_t S, int64_t S_max) {
+    LOKI_REQUIRE(S >= 1, LOKI_ERR_INVALID_ARG, "S must be >= 1 (got %lld)", (long long)S);
+    LOKI_REQUIRE(S <= S_max, LOKI_ERR_INVALID_ARG, "S (%lld) must be <= S_max (%lld)",
+                 (long long)S, (long long)S_max);
+    LOKI_REQUIRE(S <= kMaxS, LOKI_ERR_UNSUPPORTED, "S must be < 2^31 (int32 token indices)");
+    return LOKI_OK;
+}
+
+#define LOKI_CHECK(expr)                    \
+    do {                                    \
+        loki_status st_ = (expr);           \
+        if (st_ != LOKI_OK) return st_;     \
+    } while (0)
+
+#define LOKI_PTR(p, a)                                                                     \
+    do {                                                                                   \
+        LOKI_REQUIRE((p) != nullptr, LOKI_ERR_INVALID_ARG, "%s must not be NULL", #p);    \
+        LOKI_REQUIRE(aligned((p), (a)), LOKI_ERR_INVALID_ARG, "%s must be %d-byte aligned", \
+                     #p, (int)(a));                                                        \
+    } while (0)
+
+#define LOKI_CUDA(expr, where)                        \
+    do {                                              \
+        cudaError_t e_ = (expr);                      \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+loki::Dt to_dt(loki_dtype dt) { return dt == LOKI_DTYPE_F32 ? loki::kF32 : loki::kBF16; }
+
+float resolve_scale(float scale, int D) {
+    return (scale > 0.f && isfinite(scale)) ? scale : 1.0f / sqrtf((float)D);
+}
+
+// workspace pieces of the decode path
+struct DecodeWs {
+    size_t q_rot, scores, ml, acc, total;
+};
+DecodeWs decode_ws(int B, int H_q, int64_t S, int D, int64_t k) {
+    const int64_t rows = (int64_t)B * H_q;
+    const int64_t parts = loki::sparse_max_parts(k);
+    DecodeWs w;
+    w.q_rot = 0;
+    w.scores = align_up(w.q_rot + (size_t)rows * D * sizeof(float));
+    w.ml = align_up(w.scores + (size_t)rows * S * sizeof(float));
+    w.acc = align_up(w.ml + (size_t)rows * parts * sizeof(float2));
+    w.total = align_up(w.acc + (size_t)rows * parts * D * sizeof(float));
+    return w;
+}
+
+struct SparseWs {
+    size_t ml, acc, total;
+};
+SparseWs sparse_ws(int B, int H_q, int64_t k, int D) {
+    const int64_t rows = (int64_t)B * H_q;
+    const int64_t parts = loki::sparse_max_parts(k);
+    SparseWs w;
+    w.ml = 0;
+    w.acc = align_up((size_t)rows * parts * sizeof(float2));
+    w.total = align_up(w.acc + (size_t)rows * parts * D * sizeof(float));
+    return w;
+}
+
+struct DenseWs {
+    size_t ml, acc, total;
+};
+DenseWs dense_ws(int B, int H_q, int64_t S, int D) {
+    // slots: units (B * H_kv) x parts x G = B * H_q x parts
+    const int64_t slots = (int64_t)B * H_q * loki::dense_max_parts(S);
+    DenseWs w;
+    w.ml = 0;
+    w.acc = align_up((size_t)slots * sizeof(float2));
+    w.total = align_up(w.acc + (size_t)slots * D * sizeof(float));
+    return w;
+}
+
+struct CalWs {
+    size_t mean, cov, vec, total;
+};
+CalWs cal_ws(int H_kv, int D) {
+    CalWs w;
+    w.mean = 0;
+    w.cov = align_up((size_t)H_kv * D * sizeof(double));
+    w.vec = align_up(w.cov + (size_t)H_kv * D * D * sizeof(double));
+    w.total = align_up(w.vec + (size_t)H_kv * D * D * sizeof(double));
+    return w;
+}
+
+template <class T>
+T* at(void* base, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* loki_status_string(loki_status st) {
+    switch (st) {
+        case LOKI_OK: return "LOKI_OK";
+        case LOKI_ERR_INVALID_ARG: return "LOKI_ERR_INVALID_ARG: invalid argument";
+        case LOKI_ERR_UNSUPPORTED: return "LOKI_ERR_UNSUPPORTED: unsupported configuration";
+        case LOKI_ERR_WORKSPACE_TOO_SMALL: return "LOKI_ERR_WORKSPACE_TOO_SMALL: workspace too small";
+        case LOKI_ERR_CUDA: return "LOKI_ERR_CUDA: CUDA runtime error";
+    }
+    return "unknown loki_status";
+}
+
+const char* loki_last_error(void) { return g_last_error.c_str(); }
+
+// ---------------------------------------------------------------------------
+
+size_t loki_calibrate_workspace_size(int64_t N, int H_kv, int D) {
+    (void)N;
+    if (H_kv < 1 || D < 1) return 0;
+    return cal_ws(H_kv, D).total;
+}
+
+loki_status loki_calibrate_pca(const void* keys, loki_dtype dt, int64_t N, int H_kv, int D,
+                               float* P, float* eigvals, void* ws, size_t ws_bytes,
+                               void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_REQUIRE(N >= 2, LOKI_ERR_INVALID_ARG, "N must be >= 2 (got %lld)", (long long)N);
+    LOKI_REQUIRE(H_kv >= 1 && H_kv <= 65535, LOKI_ERR_INVALID_ARG, "H_kv must be in [1, 65535]");
+    LOKI_REQUIRE(D >= 16 && D <= 128 && D % 16 == 0, LOKI_ERR_UNSUPPORTED,
+                 "calibration supports D in {16, 32, ..., 128} (got %d)", D);
+    LOKI_PTR(keys, 16);
+    LOKI_PTR(P, 16);
+    if (eigvals) LOKI_PTR(eigvals, 4);
+    LOKI_PTR(ws, 256);
+    const CalWs w = cal_ws(H_kv, D);
+    LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, w.total);
+    LOKI_CUDA(loki::launch_calibrate(to_dt(dt), keys, N, H_kv, D, P, eigvals, at<double>(ws, w.mean),
+                                     at<double>(ws, w.cov), at<double>(ws, w.vec),
+                                     static_cast<cudaStream_t>(stream)),
+              "loki_calibrate_pca");
+    return LOKI_OK;
+}
+
+loki_status loki_append_keys(const void* K_new, const void* V_new, const float* P,
+                             void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
+                             int64_t S_max, int64_t pos, loki_dtype dt, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_kv, H_kv, D));
+    LOKI_REQUIRE(T >= 1, LOKI_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    LOKI_REQUIRE(pos >= 0 && S_max >= 1 && pos + T <= S_max, LOKI_ERR_INVALID_ARG,
+                 "need 0 <= pos and pos + T <= S_max (pos %lld, T %d, S_max %lld)",
+                 (long long)pos, T, (long long)S_max);
+    LOKI_PTR(K_new, 16);
+    LOKI_PTR(V_new, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_CUDA(loki::launch_append(to_dt(dt), K_new, V_new, P, Kt_cache, V_cache, B, H_kv, T, D,
+                                  S_max, pos, static_cast<cudaStream_t>(stream)),
+              "loki_append_keys");
+    return LOKI_OK;
+}
+
+// ---------------------------------------------------------------------------
+
+size_t loki_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, int D, int d, int64_t k) {
+    (void)H_kv;
+    (void)d;
+    if (B < 1 || H_q < 1 || S < 1 || D < 1 || k < 1) return 0;
+    return decode_ws(B, H_q, S, D, k).total;
+}
+
+static loki_status check_decode_common(int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D,
+                                       loki_dtype dt) {
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_q, H_kv, D));
+    LOKI_CHECK(check_seq(S, S_max));
+    return LOKI_OK;
+}
+
+loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
+                                  const float* P, int B, int H_q, int H_kv, int64_t S,
+                                  int64_t S_max, int D, int d, int64_t k, float scale,
+                                  loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
+    LOKI_REQUIRE(k >= 1 && k <= S, LOKI_ERR_INVALID_ARG, "k must be in [1, S] (got %lld)",
+                 (long long)k);
+    LOKI_PTR(q, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_PTR(ws, 256);
+    const DecodeWs w = decode_ws(B, H_q, S, D, k);
+    LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, w.total);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const loki::Dt t = to_dt(dt);
+    float* q_rot = at<float>(ws, w.q_rot);
+    float* scores = at<float>(ws, w.scores);
+    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), "project_query");
+    LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, d, scores, s),
+              "score_lowdim");
+    LOKI_CUDA(loki::launch_topk(scores, (int64_t)B * H_q, S, k, selected_idx, s), "topk");
+    LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
+                                            S, S_max, D, k, resolve_scale(scale, D), out,
+                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), s),
+              "sparse_attention");
+    return LOKI_OK;
+}
+
+loki_status loki_project_query(const void* q, const float* P, int B, int H_q, int H_kv, int D,
+                               loki_dtype dt, float* q_rot, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_q, H_kv, D));
+    LOKI_PTR(q, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(q_rot, 16);
+    LOKI_CUDA(loki::launch_project_query(to_dt(dt), q, P, B, H_q, H_kv, D, q_rot,
+                                         static_cast<cudaStream_t>(stream)),
+              "project_query");
+    return LOKI_OK;
+}
+
+loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, int H_q, int H_kv,
+                              int64_t S, int64_t S_max, int D, int d, loki_dtype dt,
+                              float* scores, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
+    LOKI_PTR(q_rot, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(scores, 4);
+    LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, d,
+                                        scores, static_cast<cudaStream_t>(stream)),
+              "score_lowdim");
+    return LOKI_OK;
+}
+
+size_t loki_topk_workspace_size(int64_t rows, int64_t S, int64_t k) {
+    (void)rows;
+    (void)S;
+    (void)k;
+    return 0;
+}
+
+loki_status loki_topk(const float* scores, int64_t rows, int64_t S, int64_t k,
+                      int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    (void)ws;
+    (void)ws_bytes;
+    LOKI_REQUIRE(rows >= 1 && rows <= 0x7fffffff, LOKI_ERR_INVALID_ARG,
+                 "rows must be in [1, 2^31) (got %lld)", (long long)rows);
+    LOKI_REQUIRE(S >= 1 && S <= kMaxS, LOKI_ERR_INVALID_ARG, "S must be in [1, 2^31)");
+    LOKI_REQUIRE(k >= 1 && k <= S, LOKI_ERR_INVALID_ARG, "k must be in [1, S] (got %lld)",
+                 (long long)k);
+    LOKI_PTR(scores, 4);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_CUDA(loki::launch_topk(scores, rows, S, k, selected_idx, static_cast<cudaStream_t>(stream)),
+              "topk");
+    return LOKI_OK;
+}
+
+size_t loki_sparse_attention_workspace_size(int B, int H_q, int64_t k, int D) {
+    if (B < 1 || H_q < 1 || k < 1 || D < 1) return 0;
+    return sparse_ws(B, H_q, k, D).total;
+}
+
+loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, const void* V_cache,
+                                  const int32_t* selected_idx, int B, int H_q, int H_kv,
+                                  int64_t S, int64_t S_max, int D, int64_t k, float scale,
+                                  loki_dtype dt, void* out, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_REQUIRE(k >= 1 && k <= kMaxS, LOKI_ERR_INVALID_ARG, "k must be in [1, 2^31)");
+    LOKI_PTR(q_rot, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(ws, 256);
+    const SparseWs w = sparse_ws(B, H_q, k, D);
+    LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, w.total);
+    LOKI_CUDA(loki::launch_sparse_attention(to_dt(dt), q_rot, Kt_cache, V_cache, selected_idx, B,
+                                            H_q, H_kv, S, S_max, D, k, resolve_scale(scale, D), out,
+                                            at<float2>(ws, w.ml), at<float>(ws, w.acc),
+                                            static_cast<cudaStream_t>(stream)),
+              "sparse_attention");
+    return LOKI_OK;
+}
+
+// ---------------------------------------------------------------------------
+
+size_t dense_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, int D) {
+    (void)H_kv;
+    if (B < 1 || H_q < 1 || S < 1 || D < 1) return 0;
+    return dense_ws(B, H_q, S, D).total;
+}
+
+loki_status dense_decode_attention(const void* q, const void* K_cache, const void* V_cache,
+                                   int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D,
+                                   float scale, loki_dtype dt, void* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_PTR(q, 16);
+    LOKI_PTR(K_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(ws, 256);
+    const DenseWs w = dense_ws(B, H_q, S, D);
+    LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, w.total);
+    LOKI_CUDA(loki::launch_dense(to_dt(dt), q, K_cache, V_cache, B, H_q, H_kv, S, S_max, D,
+                                 resolve_scale(scale, D), out, at<float2>(ws, w.ml),
+                                 at<float>(ws, w.acc), static_cast<cudaStream_t>(stream)),
+              "dense_decode_attention");
+    return LOKI_OK;
+}
+
+}  // extern "C"

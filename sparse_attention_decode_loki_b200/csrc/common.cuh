@@ -1,0 +1,81 @@
+// Shared device helpers for the Loki sm_100a kernels: 16-byte loads, element
+// unpacking, warp reductions and the per-device launch-shape cache.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace loki {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 16-byte read-only load that does not allocate in L1 (each byte is used once).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 word.
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Element traits: how many elements one 16-byte vector holds and how to unpack it.
+struct ElemF32 {
+    using T = float;
+    static constexpr int kVec = 4;
+    static constexpr int kBytes = 4;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static float load1(const T* p) { return *p; }
+    __device__ __forceinline__ static T from_float(float x) { return x; }
+};
+
+struct ElemBF16 {
+    using T = __nv_bfloat16;
+    static constexpr int kVec = 8;
+    static constexpr int kBytes = 2;
+    __device__ __forceinline__ static void unpack(const uint4& v, float* f) {
+        f[0] = bf16_lo(v.x);
+        f[1] = bf16_hi(v.x);
+        f[2] = bf16_lo(v.y);
+        f[3] = bf16_hi(v.y);
+        f[4] = bf16_lo(v.z);
+        f[5] = bf16_hi(v.z);
+        f[6] = bf16_lo(v.w);
+        f[7] = bf16_hi(v.w);
+    }
+    __device__ __forceinline__ static float load1(const T* p) { return __bfloat162float(*p); }
+    __device__ __forceinline__ static T from_float(float x) { return __float2bfloat16_rn(x); }
+};
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+template <int W>
+__device__ __forceinline__ float group_sum(float v) {
+    // butterfly over the W lanes of an aligned group (W a power of two <= 32)
+#pragma unroll
+    for (int off = W / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+__device__ __forceinline__ float group_sum_rt(float v, int w) {
+    for (int off = w >> 1; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// Stream-K style static split of `total` work items over `grid` CTAs: CTA c
+// owns items [c * per, min((c + 1) * per, total)).
+struct Split {
+    int64_t total;
+    int64_t per;
+};
+
+}  // namespace loki

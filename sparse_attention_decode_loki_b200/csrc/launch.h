@@ -1,0 +1,57 @@
+// Internal host-side launchers, one per kernel family. The C ABI (api.cu)
+// validates arguments, carves workspaces and calls these; each returns the
+// CUDA error of its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace loki {
+
+enum Dt : int { kF32 = 0, kBF16 = 1 };
+
+// number of SMs and opt-in shared memory of the current device (cached)
+struct DevInfo {
+    int device;
+    int sm_count;
+    int smem_optin;
+};
+cudaError_t dev_info(DevInfo* out);
+
+// resident CTAs per SM of `func` at `threads` threads and `smem` dynamic bytes (cached)
+int occupancy(const void* func, int threads, size_t smem);
+
+// ---- decode steps --------------------------------------------------------
+cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
+                                 int D, float* q_rot, cudaStream_t s);
+
+cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B, int H_q,
+                                int H_kv, int64_t S, int64_t S_max, int D, int d, float* scores,
+                                cudaStream_t s);
+
+cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
+                        cudaStream_t s);
+
+// split-k partial slots per (batch, query head) row
+int64_t sparse_max_parts(int64_t k);
+cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
+                                    const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
+                                    int64_t S_max, int D, int64_t k, float scale, void* out,
+                                    float2* part_ml, float* part_acc, cudaStream_t s);
+
+// split-S partial slots per (batch, KV head) unit
+int64_t dense_max_parts(int64_t S);
+cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int B, int H_q,
+                         int H_kv, int64_t S, int64_t S_max, int D, float scale, void* out,
+                         float2* part_ml, float* part_acc, cudaStream_t s);
+
+// ---- supporting subsystems -----------------------------------------------
+cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
+                          void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
+                          int64_t S_max, int64_t pos, cudaStream_t s);
+
+cudaError_t launch_calibrate(Dt dt, const void* keys, int64_t N, int H_kv, int D, float* P,
+                             float* eigvals, double* ws_mean, double* ws_cov, double* ws_vec,
+                             cudaStream_t s);
+
+}  // namespace loki
