@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="run a few untimed decode, dense and append steps on seeded random "
+                         "full-size buffers (a small, allocation-light program for ncu)")
     return ap.parse_args()
 
 
@@ -477,8 +480,36 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_ncu_case(args):
+    """Each hot-path kernel a few times on the workload's full-size buffers, nothing timed."""
+    import torch
+
+    import sparse_attention_decode_loki_b200 as loki
+    import workloads
+    wl = workloads.get(args.workload)
+    dev = torch.device("cuda", 0)
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed)
+    Kt = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
+    V = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
+    q = torch.randn((wl.B, wl.H_q, wl.D), generator=g, device=dev, dtype=dt)
+    P = torch.linalg.qr(torch.randn((wl.H_kv, wl.D, wl.D), generator=g, device=dev))[0].contiguous()
+    for _ in range(max(1, args.steps)):
+        loki.loki_decode_attention(q, Kt, V, P, wl.S, wl.d, wl.k, wl.scale)
+    for _ in range(2):
+        loki.dense_decode_attention(q, Kt, V, wl.S, wl.scale)
+    Kc = torch.empty((wl.B, wl.H_kv, 8, wl.D), dtype=dt, device=dev)
+    loki.loki_append_keys(Kt[:, :, :1].contiguous(), V[:, :, :1].contiguous(), P, Kc,
+                          torch.empty_like(Kc), 0)
+    torch.cuda.synchronize()
+
+
 def main():
     args = parse_args()
+    if args.ncu_case:
+        run_ncu_case(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -56,7 +56,7 @@ def host_inputs(wl: workloads.Workload) -> HostInputs:
         P, w = oracle.calibrate_pca(g["K_cal"][:, h, :])
         Ps.append(P)
         eigs.append(w)
-    P32 = np.stack(Ps).astype(np.float32)
+    P32 = np.ascontiguousarray(np.stack(Ps), dtype=np.float32)
     Kt = np.empty_like(g["K"])
 
     def rot(bh):
