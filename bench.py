@@ -243,17 +243,19 @@ def build_gpu_inputs(wl, dev, rank):
     S_max = wl.S
     Kt = torch.empty((wl.B, wl.H_kv, S_max, wl.D), dtype=dt, device=dev)
     V = torch.empty_like(Kt)
+    # low-dimensional key plane: a contiguous copy of the first d rotated columns
+    Kt_lo = torch.empty((wl.B, wl.H_kv, S_max, wl.d), dtype=dt, device=dev)
     K_raw = torch.from_numpy(g.pop("K")).to(dev).to(dt)
     V_raw = torch.from_numpy(g.pop("V")).to(dev).to(dt)
-    loki.loki_append_keys(K_raw, V_raw, P, Kt, V, 0)
+    loki.loki_append_keys(K_raw, V_raw, P, Kt, V, 0, Kt_lo=Kt_lo)
     # the new token of the timed append (one per sequence and KV head)
     K_new = K_raw[:, :, -1:].contiguous()
     V_new = V_raw[:, :, -1:].contiguous()
     del K_raw, V_raw
     q = torch.from_numpy(g["q"]).to(dev).to(dt)
     torch.cuda.synchronize()
-    return {"q": q, "Kt": Kt, "V": V, "P": P, "eig": eig, "K_new": K_new, "V_new": V_new,
-            "q_host": g["q"]}
+    return {"q": q, "Kt": Kt, "V": V, "Kt_lo": Kt_lo, "P": P, "eig": eig, "K_new": K_new,
+            "V_new": V_new, "q_host": g["q"]}
 
 
 def run_ours(args):
@@ -271,7 +273,7 @@ def run_ours(args):
                                 device_id=dev)
     wl = workloads.get(args.workload)
     inp = build_gpu_inputs(wl, dev, rank)
-    q, Kt, V, P = inp["q"], inp["Kt"], inp["V"], inp["P"]
+    q, Kt, V, P, Kt_lo = inp["q"], inp["Kt"], inp["V"], inp["P"], inp["Kt_lo"]
     B, H_q, H_kv, S, D, d, k = wl.B, wl.H_q, wl.H_kv, wl.S, wl.D, wl.d, wl.k
     e = wl.elem_bytes
     out = torch.empty_like(q)
@@ -282,6 +284,10 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def decode():
+        loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
+                                   workspace=ws, Kt_lo=Kt_lo)
+
+    def decode_rows_only():
         loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
                                    workspace=ws)
 
@@ -332,7 +338,7 @@ def run_ours(args):
         if ev: ev[0].record(stream)
         loki.loki_project_query(q, P, q_rot)
         if ev: ev[1].record(stream)
-        loki.loki_score_lowdim(q_rot, Kt, S, d, scores)
+        loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores)
         if ev: ev[2].record(stream)
         loki.loki_topk(scores, k, idx)
         if ev: ev[3].record(stream)
@@ -342,6 +348,9 @@ def run_ours(args):
     names = ["project_query", "score_lowdim", "topk", "sparse_attention+combine"]
     kern_us = {n: statistics.mean(e_[j].elapsed_time(e_[j + 1]) for e_ in evs) * 1e3
                for j, n in enumerate(names)}
+
+    # ---- the same step on the row-only cache layout (no low-dim plane) ---------
+    rows_only_us = statistics.mean(timed(decode_rows_only, nb, 10)) * 1e3
 
     # ---- dense baseline on the same cache (q~ rounded to the cache dtype) ------
     q_rot_dt = loki.loki_project_query(q, P).to(q.dtype)
@@ -407,11 +416,13 @@ def run_ours(args):
         "data": "synthetic (seeded low-rank keys, N(0,1) values; PCA and cache built by the library)",
         "config": {"workload": wl.name, "B": B, "H_q": H_q, "H_kv": H_kv, "D": D, "S": S,
                    "d": d, "k": k, "cache_dtype": wl.dtype,
+                   "cache_layout": "rotated K rows + contiguous d-column key plane",
                    "l2": "flushed (256 MiB write) before every timed step, flush excluded",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "tokens_per_s": round(B * world * 1e6 / us_per_step_rank, 1),
         "hbm_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
         "hbm_frac_of_" + peak_kind: round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 4),
+        "rows_only_layout_us": round(rows_only_us, 3),
         "dense_us": round(dense_us, 3),
         "speedup_vs_dense": round(dense_us / step_us, 3),
         "append_us": round(append_us, 3),

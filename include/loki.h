@@ -109,6 +109,19 @@ LOKI_API loki_status loki_append_keys(const void* K_new, const void* V_new, cons
                              void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
                              int64_t S_max, int64_t pos, loki_dtype dt, void* stream);
 
+/*
+ * Same append, for caches that also keep a low-dimensional key plane:
+ *   Kt_lo [B, H_kv, S_max, d_lo] (dt) receives the first d_lo rotated columns
+ *   of each new key (a copy of K~[..., :d_lo]); d_lo * sizeof(dt) must be a
+ *   multiple of 16 bytes. The plane lets the score scan read d_lo contiguous
+ *   columns per token instead of d_lo columns out of every D-column row (a
+ *   memory-layout choice of this library; the method itself is unchanged).
+ */
+LOKI_API loki_status loki_append_keys_plane(const void* K_new, const void* V_new, const float* P,
+                                            void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo,
+                                            int B, int H_kv, int T, int D, int64_t S_max,
+                                            int64_t pos, loki_dtype dt, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention (the per-step hot path)                                 */
 /* ------------------------------------------------------------------------ */
@@ -133,6 +146,20 @@ LOKI_API loki_status loki_decode_attention(const void* q, const void* Kt_cache, 
                                   loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/*
+ * loki_decode_attention over a cache that also holds a low-dimensional key
+ * plane Kt_lo [B, H_kv, S_max, d_lo] (filled by loki_append_keys_plane):
+ * identical results; the score scan reads the plane. Requires d <= d_lo.
+ * Same workspace size as loki_decode_attention.
+ */
+LOKI_API loki_status loki_decode_attention_plane(const void* q, const void* Kt_cache,
+                                                 const void* V_cache, const void* Kt_lo, int d_lo,
+                                                 const float* P, int B, int H_q, int H_kv,
+                                                 int64_t S, int64_t S_max, int D, int d, int64_t k,
+                                                 float scale, loki_dtype dt, void* out,
+                                                 int32_t* selected_idx, void* ws, size_t ws_bytes,
+                                                 void* stream);
+
 /* Steps of loki_decode_attention, callable one by one ------------------- */
 
 /* q_rot [B, H_q, D] fp32 = q P (query rotated into its KV head's basis). */
@@ -142,7 +169,9 @@ LOKI_API loki_status loki_project_query(const void* q, const float* P, int B, in
 /*
  * scores [B, H_q, S] fp32: s_j = sum_{i<d} q_rot[i] K~_j[i] for j < S. Only
  * the first d columns of each cached key are read; each KV head's rows are
- * read once for all of its query heads.
+ * read once for all of its query heads. Kt_cache rows hold D elements: the
+ * rotated cache (D = 128) or a low-dimensional key plane (D = d_lo, with
+ * D * sizeof(dt) a multiple of 16 bytes); 1 <= d <= D. q_rot is [B, H_q, 128].
  */
 LOKI_API loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, int H_q, int H_kv,
                               int64_t S, int64_t S_max, int D, int d, loki_dtype dt,

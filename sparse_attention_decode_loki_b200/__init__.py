@@ -22,6 +22,7 @@ from ._lib import DTYPE_BF16, DTYPE_F32, LIB_PATH, LokiError, check, lib  # noqa
 __all__ = [
     "LokiError", "LIB_PATH",
     "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
+    "loki_append_keys_plane", "loki_decode_attention_plane",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
     "loki_sparse_attention_workspace_size", "loki_calibrate_workspace_size",
@@ -110,8 +111,13 @@ def loki_calibrate_pca(keys: torch.Tensor, P: Optional[torch.Tensor] = None,
 
 
 def loki_append_keys(K_new: torch.Tensor, V_new: torch.Tensor, P: torch.Tensor,
-                     Kt_cache: torch.Tensor, V_cache: torch.Tensor, pos: int) -> None:
-    """Rotate K_new [B, H_kv, T, D] by P and write it, with V_new, into cache rows [pos, pos+T)."""
+                     Kt_cache: torch.Tensor, V_cache: torch.Tensor, pos: int,
+                     Kt_lo: Optional[torch.Tensor] = None) -> None:
+    """Rotate K_new [B, H_kv, T, D] by P and write it, with V_new, into cache rows [pos, pos+T).
+
+    With Kt_lo [B, H_kv, S_max, d_lo] the first d_lo rotated columns also go to
+    that low-dimensional key plane (loki_append_keys_plane).
+    """
     dev = _cuda(K_new, V_new, P, Kt_cache, V_cache)
     B, H_kv, T, D = K_new.shape
     S_max = Kt_cache.shape[2]
@@ -124,9 +130,27 @@ def loki_append_keys(K_new: torch.Tensor, V_new: torch.Tensor, P: torch.Tensor,
             raise TypeError("K_new, V_new and the caches must share a dtype")
     if P.dtype != torch.float32 or tuple(P.shape) != (H_kv, D, D):
         raise ValueError("P must be float32 [H_kv, D, D]")
-    check(lib.loki_append_keys(K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
-                               Kt_cache.data_ptr(), V_cache.data_ptr(), B, H_kv, T, D, S_max, pos,
-                               _dt(K_new), _stream(dev)), "loki_append_keys")
+    if Kt_lo is None:
+        check(lib.loki_append_keys(K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+                                   Kt_cache.data_ptr(), V_cache.data_ptr(), B, H_kv, T, D, S_max,
+                                   pos, _dt(K_new), _stream(dev)), "loki_append_keys")
+        return
+    _check_plane(Kt_lo, Kt_cache)
+    check(lib.loki_append_keys_plane(K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+                                     Kt_cache.data_ptr(), V_cache.data_ptr(), Kt_lo.data_ptr(),
+                                     Kt_lo.shape[3], B, H_kv, T, D, S_max, pos, _dt(K_new),
+                                     _stream(dev)), "loki_append_keys_plane")
+
+
+def loki_append_keys_plane(K_new, V_new, P, Kt_cache, V_cache, Kt_lo, pos: int) -> None:
+    """loki_append_keys that also fills the low-dimensional key plane Kt_lo."""
+    loki_append_keys(K_new, V_new, P, Kt_cache, V_cache, pos, Kt_lo=Kt_lo)
+
+
+def _check_plane(Kt_lo: torch.Tensor, Kt_cache: torch.Tensor) -> None:
+    _cuda(Kt_lo, Kt_cache)
+    if Kt_lo.dim() != 4 or Kt_lo.shape[:3] != Kt_cache.shape[:3] or Kt_lo.dtype != Kt_cache.dtype:
+        raise ValueError("Kt_lo must be [B, H_kv, S_max, d_lo] with the cache's dtype")
 
 
 def _check_decode(q, Kt, V, P=None):
@@ -146,9 +170,14 @@ def loki_decode_attention(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torc
                           P: torch.Tensor, S: int, d: int, k: int, scale: float = 0.0,
                           out: Optional[torch.Tensor] = None,
                           selected_idx: Optional[torch.Tensor] = None,
-                          workspace: Optional[torch.Tensor] = None
+                          workspace: Optional[torch.Tensor] = None,
+                          Kt_lo: Optional[torch.Tensor] = None
                           ) -> Tuple[torch.Tensor, torch.Tensor]:
-    """One Loki decode step. Returns (out [B, H_q, D], selected_idx [B, H_q, k] int32)."""
+    """One Loki decode step. Returns (out [B, H_q, D], selected_idx [B, H_q, k] int32).
+
+    With Kt_lo (a low-dimensional key plane filled by loki_append_keys_plane)
+    the score scan reads the plane (loki_decode_attention_plane).
+    """
     dev, B, H_q, H_kv, S_max, D = _check_decode(q, Kt_cache, V_cache, P)
     if out is None:
         out = torch.empty_like(q)
@@ -156,11 +185,29 @@ def loki_decode_attention(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torc
         selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
     _cuda(q, out, selected_idx)
     ws = _ws(loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k), dev, workspace)
-    check(lib.loki_decode_attention(q.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
-                                    P.data_ptr(), B, H_q, H_kv, S, S_max, D, d, k, float(scale),
-                                    _dt(q), out.data_ptr(), selected_idx.data_ptr(), ws.data_ptr(),
-                                    _ws_bytes(ws), _stream(dev)), "loki_decode_attention")
+    if Kt_lo is None:
+        check(lib.loki_decode_attention(q.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
+                                        P.data_ptr(), B, H_q, H_kv, S, S_max, D, d, k,
+                                        float(scale), _dt(q), out.data_ptr(),
+                                        selected_idx.data_ptr(), ws.data_ptr(), _ws_bytes(ws),
+                                        _stream(dev)), "loki_decode_attention")
+    else:
+        _check_plane(Kt_lo, Kt_cache)
+        check(lib.loki_decode_attention_plane(q.data_ptr(), Kt_cache.data_ptr(),
+                                              V_cache.data_ptr(), Kt_lo.data_ptr(),
+                                              Kt_lo.shape[3], P.data_ptr(), B, H_q, H_kv, S, S_max,
+                                              D, d, k, float(scale), _dt(q), out.data_ptr(),
+                                              selected_idx.data_ptr(), ws.data_ptr(),
+                                              _ws_bytes(ws), _stream(dev)),
+              "loki_decode_attention_plane")
     return out, selected_idx
+
+
+def loki_decode_attention_plane(q, Kt_cache, V_cache, Kt_lo, P, S: int, d: int, k: int,
+                                scale: float = 0.0, out=None, selected_idx=None, workspace=None):
+    """loki_decode_attention scoring from the low-dimensional key plane Kt_lo."""
+    return loki_decode_attention(q, Kt_cache, V_cache, P, S, d, k, scale, out, selected_idx,
+                                 workspace, Kt_lo=Kt_lo)
 
 
 def loki_project_query(q: torch.Tensor, P: torch.Tensor,

@@ -30,10 +30,17 @@ PROTOTYPES = {
                                    c_void_p, c_size_t, c_void_p]),
     "loki_append_keys": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                  c_int, c_int, c_int64, c_int64, c_int, c_void_p]),
+    "loki_append_keys_plane": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_int, c_int, c_int, c_int, c_int, c_int64, c_int64, c_int,
+                                       c_void_p]),
     "loki_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int64, c_int, c_int, c_int64]),
     "loki_decode_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                       c_int64, c_int64, c_int, c_int, c_int64, c_float, c_int,
                                       c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "loki_decode_attention_plane": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                            c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,
+                                            c_int, c_int64, c_float, c_int, c_void_p, c_void_p,
+                                            c_void_p, c_size_t, c_void_p]),
     "loki_project_query": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p,
                                    c_void_p]),
     "loki_score_lowdim": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,

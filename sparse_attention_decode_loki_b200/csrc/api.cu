@@ -68,6 +68,15 @@ loki_status check_seq(int64_t S, int64_t S_max) {
     return LOKI_OK;
 }
 
+loki_status check_plane(int d_lo, int D, loki_dtype dt) {
+    const int e = dt == LOKI_DTYPE_F32 ? 4 : 2;
+    LOKI_REQUIRE(d_lo >= 1 && d_lo <= D, LOKI_ERR_INVALID_ARG, "d_lo must be in [1, D] (got %d)",
+                 d_lo);
+    LOKI_REQUIRE((d_lo * e) % 16 == 0, LOKI_ERR_INVALID_ARG,
+                 "d_lo * element size must be a multiple of 16 bytes (got d_lo = %d)", d_lo);
+    return LOKI_OK;
+}
+
 #define LOKI_CHECK(expr)                    \
     do {                                    \
         loki_status st_ = (expr);           \
@@ -215,9 +224,33 @@ loki_status loki_append_keys(const void* K_new, const void* V_new, const float* 
     LOKI_PTR(P, 16);
     LOKI_PTR(Kt_cache, 16);
     LOKI_PTR(V_cache, 16);
-    LOKI_CUDA(loki::launch_append(to_dt(dt), K_new, V_new, P, Kt_cache, V_cache, B, H_kv, T, D,
-                                  S_max, pos, static_cast<cudaStream_t>(stream)),
+    LOKI_CUDA(loki::launch_append(to_dt(dt), K_new, V_new, P, Kt_cache, V_cache, nullptr, 0, B,
+                                  H_kv, T, D, S_max, pos, static_cast<cudaStream_t>(stream)),
               "loki_append_keys");
+    return LOKI_OK;
+}
+
+loki_status loki_append_keys_plane(const void* K_new, const void* V_new, const float* P,
+                                   void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B,
+                                   int H_kv, int T, int D, int64_t S_max, int64_t pos,
+                                   loki_dtype dt, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_kv, H_kv, D));
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    LOKI_REQUIRE(T >= 1, LOKI_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    LOKI_REQUIRE(pos >= 0 && S_max >= 1 && pos + T <= S_max, LOKI_ERR_INVALID_ARG,
+                 "need 0 <= pos and pos + T <= S_max (pos %lld, T %d, S_max %lld)",
+                 (long long)pos, T, (long long)S_max);
+    LOKI_PTR(K_new, 16);
+    LOKI_PTR(V_new, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(Kt_lo, 16);
+    LOKI_CUDA(loki::launch_append(to_dt(dt), K_new, V_new, P, Kt_cache, V_cache, Kt_lo, d_lo, B,
+                                  H_kv, T, D, S_max, pos, static_cast<cudaStream_t>(stream)),
+              "loki_append_keys_plane");
     return LOKI_OK;
 }
 
@@ -238,11 +271,11 @@ static loki_status check_decode_common(int B, int H_q, int H_kv, int64_t S, int6
     return LOKI_OK;
 }
 
-loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
-                                  const float* P, int B, int H_q, int H_kv, int64_t S,
-                                  int64_t S_max, int D, int d, int64_t k, float scale,
-                                  loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
-                                  size_t ws_bytes, void* stream) {
+static loki_status decode_impl(const char* name, const void* q, const void* Kt_cache,
+                               const void* V_cache, const void* Kt_lo, int d_lo, const float* P,
+                               int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                               int64_t k, float scale, loki_dtype dt, void* out,
+                               int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream) {
     g_last_error.clear();
     LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
     LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
@@ -255,6 +288,11 @@ loki_status loki_decode_attention(const void* q, const void* Kt_cache, const voi
     LOKI_PTR(out, 16);
     LOKI_PTR(selected_idx, 4);
     LOKI_PTR(ws, 256);
+    if (Kt_lo != nullptr) {
+        LOKI_CHECK(check_plane(d_lo, D, dt));
+        LOKI_PTR(Kt_lo, 16);
+        LOKI_REQUIRE(d <= d_lo, LOKI_ERR_INVALID_ARG, "d (%d) must be <= d_lo (%d)", d, d_lo);
+    }
     const DecodeWs w = decode_ws(B, H_q, S, D, k);
     LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
                  "workspace %zu bytes < required %zu", ws_bytes, w.total);
@@ -262,15 +300,47 @@ loki_status loki_decode_attention(const void* q, const void* Kt_cache, const voi
     const loki::Dt t = to_dt(dt);
     float* q_rot = at<float>(ws, w.q_rot);
     float* scores = at<float>(ws, w.scores);
-    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), "project_query");
-    LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, d, scores, s),
-              "score_lowdim");
-    LOKI_CUDA(loki::launch_topk(scores, (int64_t)B * H_q, S, k, selected_idx, s), "topk");
+    // The first kernel is ordered normally after whatever precedes the call;
+    // the later ones use programmatic dependent launch.
+    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), name);
+    if (Kt_lo != nullptr)
+        LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
+                                            scores, s, true),
+                  name);
+    else
+        LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, D, d,
+                                            scores, s, true),
+                  name);
+    LOKI_CUDA(loki::launch_topk(scores, (int64_t)B * H_q, S, k, selected_idx, s, true), name);
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
-                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), s),
-              "sparse_attention");
+                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), s, true),
+              name);
     return LOKI_OK;
+}
+
+loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
+                                  const float* P, int B, int H_q, int H_kv, int64_t S,
+                                  int64_t S_max, int D, int d, int64_t k, float scale,
+                                  loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    return decode_impl("loki_decode_attention", q, Kt_cache, V_cache, nullptr, 0, P, B, H_q, H_kv,
+                       S, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes, stream);
+}
+
+loki_status loki_decode_attention_plane(const void* q, const void* Kt_cache, const void* V_cache,
+                                        const void* Kt_lo, int d_lo, const float* P, int B,
+                                        int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                                        int64_t k, float scale, loki_dtype dt, void* out,
+                                        int32_t* selected_idx, void* ws, size_t ws_bytes,
+                                        void* stream) {
+    if (Kt_lo == nullptr) {
+        g_last_error = "Kt_lo must not be NULL";
+        return LOKI_ERR_INVALID_ARG;
+    }
+    return decode_impl("loki_decode_attention_plane", q, Kt_cache, V_cache, Kt_lo, d_lo, P, B,
+                       H_q, H_kv, S, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes,
+                       stream);
 }
 
 loki_status loki_project_query(const void* q, const float* P, int B, int H_q, int H_kv, int D,
@@ -291,14 +361,19 @@ loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, i
                               int64_t S, int64_t S_max, int D, int d, loki_dtype dt,
                               float* scores, void* stream) {
     g_last_error.clear();
-    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_CHECK(check_dtype(dt));
+    // Kt_cache rows hold D elements: the rotated cache (D = 128) or a
+    // low-dimensional key plane (D = d_lo); q_rot rows always hold 128.
+    LOKI_CHECK(check_heads(B, H_q, H_kv, 128));
+    LOKI_CHECK(check_seq(S, S_max));
+    LOKI_CHECK(check_plane(D, 128, dt));
     LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
     LOKI_PTR(q_rot, 16);
     LOKI_PTR(Kt_cache, 16);
     LOKI_PTR(scores, 4);
-    LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, d,
-                                        scores, static_cast<cudaStream_t>(stream)),
-              "score_lowdim");
+    LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, 128, D,
+                                        d, scores, static_cast<cudaStream_t>(stream), false),
+              "loki_score_lowdim");
     return LOKI_OK;
 }
 
@@ -321,7 +396,8 @@ loki_status loki_topk(const float* scores, int64_t rows, int64_t S, int64_t k,
                  (long long)k);
     LOKI_PTR(scores, 4);
     LOKI_PTR(selected_idx, 4);
-    LOKI_CUDA(loki::launch_topk(scores, rows, S, k, selected_idx, static_cast<cudaStream_t>(stream)),
+    LOKI_CUDA(loki::launch_topk(scores, rows, S, k, selected_idx, static_cast<cudaStream_t>(stream),
+                                false),
               "topk");
     return LOKI_OK;
 }
@@ -351,7 +427,7 @@ loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, cons
     LOKI_CUDA(loki::launch_sparse_attention(to_dt(dt), q_rot, Kt_cache, V_cache, selected_idx, B,
                                             H_q, H_kv, S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc),
-                                            static_cast<cudaStream_t>(stream)),
+                                            static_cast<cudaStream_t>(stream), false),
               "sparse_attention");
     return LOKI_OK;
 }

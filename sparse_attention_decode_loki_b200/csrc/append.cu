@@ -19,8 +19,10 @@ __global__ void __launch_bounds__(128) k_rotate_append(const typename E::T* __re
                                                        const typename E::T* __restrict__ V_new,
                                                        const float* __restrict__ P,
                                                        typename E::T* __restrict__ Kt_cache,
-                                                       typename E::T* __restrict__ V_cache, int H_kv,
-                                                       int T, int D, int64_t S_max, int64_t pos) {
+                                                       typename E::T* __restrict__ V_cache,
+                                                       typename E::T* __restrict__ Kt_lo, int d_lo,
+                                                       int H_kv, int T, int D, int64_t S_max,
+                                                       int64_t pos) {
     __shared__ float kin[kAppendTokens][128];
     const int t0 = blockIdx.x * kAppendTokens;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -44,25 +46,28 @@ __global__ void __launch_bounds__(128) k_rotate_append(const typename E::T* __re
         for (int t = 0; t < kAppendTokens; ++t) acc[t] = fmaf(kin[t][i], p, acc[t]);
     }
     for (int t = 0; t < nt; ++t) {
-        const int64_t dst = (unit * S_max + pos + t0 + t) * D + c;
-        Kt_cache[dst] = E::from_float(acc[t]);
-        V_cache[dst] = V_new[(unit * T + t0 + t) * D + c];
+        const int64_t row = unit * S_max + pos + t0 + t;
+        const typename E::T kt = E::from_float(acc[t]);
+        Kt_cache[row * D + c] = kt;
+        V_cache[row * D + c] = V_new[(unit * T + t0 + t) * D + c];
+        if (Kt_lo != nullptr && c < d_lo) Kt_lo[row * d_lo + c] = kt;
     }
 }
 
 cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
-                          void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
-                          int64_t S_max, int64_t pos, cudaStream_t s) {
+                          void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
+                          int T, int D, int64_t S_max, int64_t pos, cudaStream_t s) {
     dim3 grid((T + kAppendTokens - 1) / kAppendTokens, H_kv, B), block(128);
     if (dt == kF32)
         k_rotate_append<ElemF32><<<grid, block, 0, s>>>(
             static_cast<const float*>(K_new), static_cast<const float*>(V_new), P,
-            static_cast<float*>(Kt_cache), static_cast<float*>(V_cache), H_kv, T, D, S_max, pos);
+            static_cast<float*>(Kt_cache), static_cast<float*>(V_cache),
+            static_cast<float*>(Kt_lo), d_lo, H_kv, T, D, S_max, pos);
     else
         k_rotate_append<ElemBF16><<<grid, block, 0, s>>>(
             static_cast<const __nv_bfloat16*>(K_new), static_cast<const __nv_bfloat16*>(V_new), P,
-            static_cast<__nv_bfloat16*>(Kt_cache), static_cast<__nv_bfloat16*>(V_cache), H_kv, T,
-            D, S_max, pos);
+            static_cast<__nv_bfloat16*>(Kt_cache), static_cast<__nv_bfloat16*>(V_cache),
+            static_cast<__nv_bfloat16*>(Kt_lo), d_lo, H_kv, T, D, S_max, pos);
     return cudaGetLastError();
 }
 

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(128) k_combine(const float2* __restrict__ part
     const int64_t c1 = (unit * items + items - 1) / per;
     const int np = (int)(c1 - c0 + 1);
     const int c = threadIdx.x;
+    griddep_wait();  // partials come from the attention kernel
+    griddep_launch_dependents();
     float M = -INFINITY;
     for (int p = 0; p < np; ++p) M = fmaxf(M, part_ml[(unit * maxp + p) * Gc + g].x);
     float L = 0.f, A = 0.f;

@@ -71,11 +71,40 @@ __device__ __forceinline__ float group_sum_rt(float v, int w) {
     return v;
 }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialization attribute may start while its predecessor on the
+// stream is still running; griddep_wait() blocks until the predecessor grid
+// has completed and its writes are visible (a no-op without the attribute).
+// griddep_launch_dependents() lets the next kernel be scheduled early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 // Stream-K style static split of `total` work items over `grid` CTAs: CTA c
 // owns items [c * per, min((c + 1) * per, total)).
 struct Split {
     int64_t total;
     int64_t per;
 };
+
+// Launch `kern` on `s`; with pdl the launch carries the programmatic
+// stream-serialization attribute (the kernel must griddep_wait() before
+// reading anything its predecessor writes).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 }  // namespace loki

@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
 
     const int grp = threadIdx.x / LPR;
     const int sub = threadIdx.x % LPR;
+    griddep_launch_dependents();  // lets the combine kernel be scheduled early
 
     int64_t w = (int64_t)blockIdx.x * per;
     const int64_t w_end = min64(w + per, total);
@@ -174,9 +175,9 @@ static cudaError_t dense_impl(const void* q, const void* K, const void* V, int B
                                         scale * kLog2e, total, per, maxp, part_ml, part_acc);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    k_combine<E><<<(unsigned)((int64_t)B * H_q), 128, 0, s>>>(part_ml, part_acc, static_cast<T*>(out),
-                                                             H_q, G, S, per, maxp, D);
-    return cudaGetLastError();
+    return launch_kernel(k_combine<E>, dim3((unsigned)((int64_t)B * H_q)), dim3(128), 0, s, true,
+                         (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out), H_q,
+                         G, (int64_t)S, per, maxp, D);
 }
 
 template <class E>

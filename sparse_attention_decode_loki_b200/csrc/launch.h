@@ -25,19 +25,21 @@ int occupancy(const void* func, int threads, size_t smem);
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
                                  int D, float* q_rot, cudaStream_t s);
 
+// `row` is the row length (and stride) of the key buffer scanned: D for the
+// rotated cache, d_lo for a low-dimensional key plane.
 cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B, int H_q,
-                                int H_kv, int64_t S, int64_t S_max, int D, int d, float* scores,
-                                cudaStream_t s);
+                                int H_kv, int64_t S, int64_t S_max, int D, int row, int d,
+                                float* scores, cudaStream_t s, bool pdl);
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
-                        cudaStream_t s);
+                        cudaStream_t s, bool pdl);
 
 // split-k partial slots per (batch, query head) row
 int64_t sparse_max_parts(int64_t k);
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
-                                    float2* part_ml, float* part_acc, cudaStream_t s);
+                                    float2* part_ml, float* part_acc, cudaStream_t s, bool pdl);
 
 // split-S partial slots per (batch, KV head) unit
 int64_t dense_max_parts(int64_t S);
@@ -46,9 +48,11 @@ cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int
                          float2* part_ml, float* part_acc, cudaStream_t s);
 
 // ---- supporting subsystems -----------------------------------------------
+// Kt_lo (may be null): [B, H_kv, S_max, d_lo] plane that also receives the
+// first d_lo rotated columns of each appended key.
 cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
-                          void* Kt_cache, void* V_cache, int B, int H_kv, int T, int D,
-                          int64_t S_max, int64_t pos, cudaStream_t s);
+                          void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
+                          int T, int D, int64_t S_max, int64_t pos, cudaStream_t s);
 
 cudaError_t launch_calibrate(Dt dt, const void* keys, int64_t N, int H_kv, int D, float* P,
                              float* eigvals, double* ws_mean, double* ws_cov, double* ws_vec,

@@ -16,31 +16,55 @@
 
 namespace loki {
 
-// q_rot[row, c] = sum_i q[row, i] P[h_kv, i, c]; one CTA per (batch, query head)
+// q_rot[row, c] = sum_i q[row, i] P[h_kv, i, c]. One CTA per (KV head, block of
+// 32 output columns, chunk of up to 32 query rows of that head): the P column
+// block (128 x 32 fp32) is staged once in shared memory and reused by every
+// query of the head; each warp computes one query's 32 columns per step.
+constexpr int kProjCols = 32;
+constexpr int kProjRows = 32;
+
 template <class E>
-__global__ void __launch_bounds__(128) k_project_query(const typename E::T* __restrict__ q,
+__global__ void __launch_bounds__(256) k_project_query(const typename E::T* __restrict__ q,
                                                        const float* __restrict__ P,
-                                                       float* __restrict__ q_rot, int H_q, int G,
-                                                       int D) {
-    __shared__ float qs[128];
-    const int row = blockIdx.x;
-    const int hk = (row % H_q) / G;
-    const int c = threadIdx.x;
-    if (c < D) qs[c] = E::load1(q + (int64_t)row * D + c);
+                                                       float* __restrict__ q_rot, int B, int H_q,
+                                                       int G, int D) {
+    __shared__ float Ps[128][kProjCols];
+    __shared__ float qs[kProjRows][128];
+    const int hk = blockIdx.x;
+    const int c0 = blockIdx.y * kProjCols;
+    const int r0 = blockIdx.z * kProjRows;
+    const int nrows = min(kProjRows, B * G - r0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float* Ph = P + (int64_t)hk * D * D;
+    for (int it = tid; it < D * kProjCols; it += 256) {
+        const int i = it / kProjCols, c = it % kProjCols;
+        Ps[i][c] = (c0 + c < D) ? __ldg(Ph + (int64_t)i * D + c0 + c) : 0.f;
+    }
+    // the head's queries: row j of the chunk is (batch b, group member g)
+    for (int it = tid; it < nrows * D; it += 256) {
+        const int j = it / D, i = it % D;
+        const int jr = r0 + j;
+        const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
+        qs[j][i] = E::load1(q + row * D + i);
+    }
     __syncthreads();
-    if (c >= D) return;
-    const float* Ph = P + (int64_t)hk * D * D + c;
-    float acc = 0.f;
-    for (int i = 0; i < D; ++i) acc = fmaf(qs[i], __ldg(Ph + (int64_t)i * D), acc);
-    q_rot[(int64_t)row * D + c] = acc;
+    for (int j = warp; j < nrows; j += 8) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) acc = fmaf(qs[j][i], Ps[i][lane], acc);
+        const int jr = r0 + j;
+        const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
+        if (c0 + lane < D) q_rot[row * D + c0 + lane] = acc;
+    }
 }
 
 template <class E, int G>
 __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ q_rot,
                                                       const typename E::T* __restrict__ Kt,
                                                       float* __restrict__ scores, int H_q, int H_kv,
-                                                      int S, int64_t S_max, int D, int d,
-                                                      int log2L, int64_t total, int64_t per) {
+                                                      int S, int64_t S_max, int D, int row_len,
+                                                      int d, int log2L, int64_t total,
+                                                      int64_t per) {
     constexpr int kThreads = 256;
     constexpr int U = 8;
     constexpr int KV = E::kVec;
@@ -52,7 +76,9 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
     const int rows_per_pass = kThreads >> log2L;
     const int nvec = (d + KV - 1) / KV;
     const bool lane_on = sub < nvec;
-    const int64_t row_bytes = (int64_t)D * E::kBytes;
+    const int64_t row_bytes = (int64_t)row_len * E::kBytes;
+    griddep_wait();  // q_rot comes from the projection kernel
+    griddep_launch_dependents();
 
     int64_t r = (int64_t)blockIdx.x * per;
     const int64_t r_end = min64(r + per, total);
@@ -109,20 +135,20 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
                                  int D, float* q_rot, cudaStream_t s) {
     const int G = H_q / H_kv;
-    dim3 grid(B * H_q), block(128);
+    dim3 grid(H_kv, (D + kProjCols - 1) / kProjCols, (B * G + kProjRows - 1) / kProjRows);
     if (dt == kF32)
-        k_project_query<ElemF32><<<grid, block, 0, s>>>(static_cast<const float*>(q), P, q_rot,
-                                                        H_q, G, D);
+        k_project_query<ElemF32><<<grid, 256, 0, s>>>(static_cast<const float*>(q), P, q_rot, B,
+                                                      H_q, G, D);
     else
-        k_project_query<ElemBF16><<<grid, block, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(q), P, q_rot, H_q, G, D);
+        k_project_query<ElemBF16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), P,
+                                                       q_rot, B, H_q, G, D);
     return cudaGetLastError();
 }
 
 template <class E, int G>
 static cudaError_t score_impl(const float* q_rot, const void* Kt, int B, int H_q, int H_kv,
-                              int64_t S, int64_t S_max, int D, int d, float* scores,
-                              cudaStream_t s) {
+                              int64_t S, int64_t S_max, int D, int row, int d, float* scores,
+                              cudaStream_t s, bool pdl) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
@@ -137,18 +163,19 @@ static cudaError_t score_impl(const float* q_rot, const void* Kt, int B, int H_q
     if (grid > resident) grid = resident;
     const int64_t per = (total + grid - 1) / grid;
     grid = (total + per - 1) / per;
-    kern<<<(unsigned)grid, 256, 0, s>>>(q_rot, static_cast<const typename E::T*>(Kt), scores, H_q,
-                                        H_kv, (int)S, S_max, D, d, log2L, total, per);
-    return cudaGetLastError();
+    return launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
+                         static_cast<const typename E::T*>(Kt), scores, H_q, H_kv, (int)S, S_max,
+                         D, row, d, log2L, total, per);
 }
 
 template <class E>
 static cudaError_t score_dispatch(int G, const float* q_rot, const void* Kt, int B, int H_q,
-                                  int H_kv, int64_t S, int64_t S_max, int D, int d, float* scores,
-                                  cudaStream_t s) {
+                                  int H_kv, int64_t S, int64_t S_max, int D, int row, int d,
+                                  float* scores, cudaStream_t s, bool pdl) {
     switch (G) {
 #define LOKI_G(g) \
-    case g: return score_impl<E, g>(q_rot, Kt, B, H_q, H_kv, S, S_max, D, d, scores, s);
+    case g:       \
+        return score_impl<E, g>(q_rot, Kt, B, H_q, H_kv, S, S_max, D, row, d, scores, s, pdl);
         LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
 #undef LOKI_G
         default: return cudaErrorInvalidValue;
@@ -156,12 +183,14 @@ static cudaError_t score_dispatch(int G, const float* q_rot, const void* Kt, int
 }
 
 cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B, int H_q,
-                                int H_kv, int64_t S, int64_t S_max, int D, int d, float* scores,
-                                cudaStream_t s) {
+                                int H_kv, int64_t S, int64_t S_max, int D, int row, int d,
+                                float* scores, cudaStream_t s, bool pdl) {
     const int G = H_q / H_kv;
     if (dt == kF32)
-        return score_dispatch<ElemF32>(G, q_rot, Kt, B, H_q, H_kv, S, S_max, D, d, scores, s);
-    return score_dispatch<ElemBF16>(G, q_rot, Kt, B, H_q, H_kv, S, S_max, D, d, scores, s);
+        return score_dispatch<ElemF32>(G, q_rot, Kt, B, H_q, H_kv, S, S_max, D, row, d, scores, s,
+                                       pdl);
+    return score_dispatch<ElemBF16>(G, q_rot, Kt, B, H_q, H_kv, S, S_max, D, row, d, scores, s,
+                                    pdl);
 }
 
 }  // namespace loki

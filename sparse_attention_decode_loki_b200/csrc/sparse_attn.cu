@@ -5,9 +5,11 @@
 //
 // Work items are (row, j) pairs, row = (batch, query head) and j < k the
 // position in its selected list; the B*H_q*k items are split evenly over one
-// wave of CTAs. A row group of lanes (16 lanes for bf16, 32 for fp32) owns one
-// 256/512-byte key row and the matching value row per step, with 4 rows in
-// flight; each row is a random gather, but a contiguous one. Scores use all D
+// wave of CTAs. Each CTA stages its selected indices in shared memory (1024
+// at a time), so the row gathers never wait on an index load. A row group of
+// lanes (16 lanes for bf16, 32 for fp32) owns one 256/512-byte key row and
+// the matching value row per step, with 8 rows in flight; each row is a
+// random gather, but a contiguous one. Scores use all D
 // dimensions in fp32; the softmax runs online in base 2 with the scale folded
 // into q~. Each CTA merges its row groups and writes one partial per row
 // segment; k_combine merges the partials of a row.
@@ -25,7 +27,7 @@ constexpr int kSparseMinItems = 64;  // CTAs own at least this many items
 int64_t sparse_max_parts(int64_t k) { return (k - 1) / (kSparseMinItems / 2) + 2; }
 
 template <class E>
-__global__ void __launch_bounds__(256) k_sparse_attn(
+__global__ void __launch_bounds__(256, 2) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int64_t total, int64_t per, int maxp,
@@ -34,14 +36,18 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
     constexpr int KV = E::kVec;
     constexpr int LPR = D / KV;           // lanes per row
     constexpr int NGRP = 256 / LPR;       // row groups per CTA
-    constexpr int U = 4;                  // rows in flight per group
+    constexpr int U = 8;                  // rows in flight per group
+    constexpr int kIdxChunk = 1024;       // selected indices staged per step
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
     __shared__ float sm_m[NGRP], sm_l[NGRP];
     __shared__ float sm_acc[NGRP][D];
+    __shared__ int s_idx[kIdxChunk];
 
     const int grp = threadIdx.x / LPR;
     const int sub = threadIdx.x % LPR;
     const int G = H_q / H_kv;
+    griddep_wait();  // q_rot and the selected indices come from earlier kernels
+    griddep_launch_dependents();
 
     int64_t w = (int64_t)blockIdx.x * per;
     const int64_t w_end = min64(w + per, total);
@@ -66,51 +72,59 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
 #pragma unroll
         for (int e = 0; e < KV; ++e) acc[e] = 0.f;
 
-        for (int jb = j0; jb < j1; jb += NGRP * U) {
-            int t[U];
-            uint4 kv[U], vv[U];
+        for (int cb = j0; cb < j1; cb += kIdxChunk) {
+            const int n = min(kIdxChunk, j1 - cb);
+            __syncthreads();  // the previous chunk's indices are no longer read
+            for (int t = threadIdx.x; t < n; t += 256) {
+                const int tok = __ldg(ip + cb + t);
+                s_idx[t] = ((unsigned)tok < (unsigned)S) ? tok : -1;
+            }
+            __syncthreads();
+            for (int jb = 0; jb < n; jb += NGRP * U) {
+                int t[U];
+                uint4 kv[U], vv[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int jj = jb + u * NGRP + grp;
-                int tok = jj < j1 ? __ldg(ip + jj) : -1;
-                if ((unsigned)tok >= (unsigned)S) tok = -1;
-                t[u] = tok;
-                if (tok >= 0) {
-                    kv[u] = ld_stream(Kb + (int64_t)tok * kRowBytes);
-                    vv[u] = ld_stream(Vb + (int64_t)tok * kRowBytes);
-                } else {
-                    kv[u] = make_uint4(0u, 0u, 0u, 0u);
-                    vv[u] = kv[u];
+                for (int u = 0; u < U; ++u) {
+                    const int jj = jb + u * NGRP + grp;
+                    const int tok = jj < n ? s_idx[jj] : -1;
+                    t[u] = tok;
+                    if (tok >= 0) {
+                        kv[u] = ld_stream(Kb + (int64_t)tok * kRowBytes);
+                        vv[u] = ld_stream(Vb + (int64_t)tok * kRowBytes);
+                    } else {
+                        kv[u] = make_uint4(0u, 0u, 0u, 0u);
+                        vv[u] = kv[u];
+                    }
                 }
+                float s[U];
+                float mx = m;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    float f[KV];
+                    E::unpack(kv[u], f);
+                    float a = 0.f;
+#pragma unroll
+                    for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
+                    a = group_sum<LPR>(a);
+                    s[u] = t[u] >= 0 ? a : -INFINITY;
+                    mx = fmaxf(mx, s[u]);
+                }
+                if (mx == -INFINITY) continue;
+                const float alpha = exp2f(m - mx);
+                l *= alpha;
+#pragma unroll
+                for (int e = 0; e < KV; ++e) acc[e] *= alpha;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const float p = exp2f(s[u] - mx);
+                    l += p;
+                    float f[KV];
+                    E::unpack(vv[u], f);
+#pragma unroll
+                    for (int e = 0; e < KV; ++e) acc[e] = fmaf(p, f[e], acc[e]);
+                }
+                m = mx;
             }
-            float s[U];
-            float mx = m;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                float f[KV];
-                E::unpack(kv[u], f);
-                float a = 0.f;
-#pragma unroll
-                for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
-                a = group_sum<LPR>(a);
-                s[u] = t[u] >= 0 ? a : -INFINITY;
-                mx = fmaxf(mx, s[u]);
-            }
-            if (mx == -INFINITY) continue;
-            const float alpha = exp2f(m - mx);
-            l *= alpha;
-#pragma unroll
-            for (int e = 0; e < KV; ++e) acc[e] *= alpha;
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const float p = exp2f(s[u] - mx);
-                l += p;
-                float f[KV];
-                E::unpack(vv[u], f);
-#pragma unroll
-                for (int e = 0; e < KV; ++e) acc[e] = fmaf(p, f[e], acc[e]);
-            }
-            m = mx;
         }
 
         if (sub == 0) {
@@ -147,7 +161,7 @@ template <class E>
 static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V,
                                const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                int64_t S_max, int D, int64_t k, float scale, void* out,
-                               float2* part_ml, float* part_acc, cudaStream_t s) {
+                               float2* part_ml, float* part_acc, cudaStream_t s, bool pdl) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
@@ -162,25 +176,24 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     const int maxp = (int)((k - 1) / per + 2);
     if (maxp > sparse_max_parts(k)) return cudaErrorInvalidValue;
     using T = typename E::T;
-    kern<<<(unsigned)grid, 256, 0, s>>>(q_rot, static_cast<const T*>(Kt), static_cast<const T*>(V),
-                                        idx, H_q, H_kv, (int)S, S_max, (int)k, scale * kLog2e,
-                                        total, per, maxp, part_ml, part_acc);
-    e = cudaGetLastError();
+    e = launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
+                      static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv, (int)S,
+                      S_max, (int)k, scale * kLog2e, total, per, maxp, part_ml, part_acc);
     if (e != cudaSuccess) return e;
-    k_combine<E><<<(unsigned)rows, 128, 0, s>>>(part_ml, part_acc, static_cast<T*>(out), H_q, 1,
-                                                k, per, maxp, D);
-    return cudaGetLastError();
+    return launch_kernel(k_combine<E>, dim3((unsigned)rows), dim3(128), 0, s, true,
+                         (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out), H_q,
+                         1, (int64_t)k, per, maxp, D);
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
-                                    float2* part_ml, float* part_acc, cudaStream_t s) {
+                                    float2* part_ml, float* part_acc, cudaStream_t s, bool pdl) {
     if (dt == kF32)
         return sparse_impl<ElemF32>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                    part_ml, part_acc, s);
+                                    part_ml, part_acc, s, pdl);
     return sparse_impl<ElemBF16>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                 part_ml, part_acc, s);
+                                 part_ml, part_acc, s, pdl);
 }
 
 }  // namespace loki

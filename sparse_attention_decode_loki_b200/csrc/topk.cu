@@ -3,14 +3,20 @@
 // approximate scores).
 //
 // One CTA per (batch, query head) row. Scores become order-preserving 32-bit
-// keys (larger float -> larger key; -0 folded onto +0; NaN folded onto -inf),
-// held in shared memory when the row fits. An MSB-first radix select with
-// 8-bit digits finds the k-th largest key T and how many keys equal to T
-// belong to the set; warp-aggregated shared-memory atomics keep the
-// histograms cheap when many keys share a digit. A stable compaction then
-// writes the selected indices in ascending token order, taking keys equal to
-// T from the lowest indices first. All decisions are integer compares, so the
-// result is exact and deterministic.
+// keys (larger float -> larger key; -0 folded onto +0; NaN folded onto -inf).
+// A most-significant-digit radix select finds the k-th largest key T and how
+// many keys equal to T belong to the set; a stable compaction then writes the
+// selected indices in ascending token order, taking keys equal to T from the
+// lowest indices first. All decisions are integer compares: the result is
+// exact and deterministic.
+//
+// Rows of up to 32768 keys (k_topk_reg): each thread holds a contiguous run of
+// keys in registers. The first pass histograms the top 12 key bits (4096
+// shared-memory bins, sign + exponent + 3 mantissa bits), which already
+// isolates the threshold to a narrow bin; the next passes (10 + 10 bits) only
+// touch keys inside the chosen bin, so they cost a register scan each.
+// Longer rows (k_topk_long) keep keys in shared memory, or re-read them from
+// L2 when they do not fit, with 8-bit digits and warp-aggregated atomics.
 #include "common.cuh"
 #include "launch.h"
 
@@ -51,19 +57,136 @@ __device__ __forceinline__ int block_excl_scan(int v, int* buf, int* total) {
     return before;
 }
 
+// Given per-bin counts in hist[0, nbins) (bins ordered by key), find the bin
+// holding the krem-th largest counted key. Thread t owns bins [t*per, (t+1)*per).
+// Writes the bin to *s_bin and the rank left inside it to *s_krem.
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int krem, int* buf,
+                                         int* s_bin, int* s_krem) {
+    const int per = nbins / (int)blockDim.x;
+    const int b0 = threadIdx.x * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) local += (int)hist[b0 + i];
+    int total;
+    const int before = block_excl_scan(local, buf, &total);
+    int above = total - before - local;  // keys in bins owned by higher threads
+    for (int i = per - 1; i >= 0; --i) {
+        const int c = (int)hist[b0 + i];
+        if (above < krem && above + c >= krem) {
+            *s_bin = b0 + i;
+            *s_krem = krem - above;
+        }
+        above += c;
+    }
+    __syncthreads();
+}
+
+template <int KPT, int NT>
+__global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ scores, int S, int k,
+                                                 int32_t* __restrict__ out) {
+    __shared__ uint32_t hist[4096];
+    __shared__ int scan_buf[32];
+    __shared__ int s_bin, s_krem;
+    const int tid = threadIdx.x;
+    const float* row = scores + (int64_t)blockIdx.x * S;
+    const int j0 = tid * KPT;
+    griddep_wait();  // scores come from the score kernel
+    griddep_launch_dependents();
+
+    uint32_t key[KPT];
+    if ((S & 3) == 0 && (KPT & 3) == 0) {
+#pragma unroll
+        for (int e = 0; e < KPT; e += 4) {
+            if (j0 + e < S) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(row + j0 + e));
+                key[e] = order_key(v.x);
+                key[e + 1] = order_key(v.y);
+                key[e + 2] = order_key(v.z);
+                key[e + 3] = order_key(v.w);
+            } else {
+                key[e] = key[e + 1] = key[e + 2] = key[e + 3] = 0u;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) key[e] = (j0 + e < S) ? order_key(__ldg(row + j0 + e)) : 0u;
+    }
+    // key 0 never comes from a score (NaN maps to the -inf key), so it marks
+    // padding: it is never counted, selected or histogrammed
+
+    // pass 1: top 12 bits
+    for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < KPT; ++e)
+        if (key[e]) atomicAdd(&hist[key[e] >> 20], 1u);
+    __syncthreads();
+    find_bin(hist, 4096, k, scan_buf, &s_bin, &s_krem);
+    const uint32_t bin1 = (uint32_t)s_bin;
+    int krem = s_krem;
+    __syncthreads();
+
+    // pass 2: bits 19..10 of the keys in bin1
+    for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < KPT; ++e)
+        if (key[e] && (key[e] >> 20) == bin1) atomicAdd(&hist[(key[e] >> 10) & 1023u], 1u);
+    __syncthreads();
+    find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem);
+    const uint32_t pre2 = (bin1 << 10) | (uint32_t)s_bin;
+    krem = s_krem;
+    __syncthreads();
+
+    // pass 3: bits 9..0 of the keys matching the 22-bit prefix
+    for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < KPT; ++e)
+        if (key[e] && (key[e] >> 10) == pre2) atomicAdd(&hist[key[e] & 1023u], 1u);
+    __syncthreads();
+    find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem);
+    const uint32_t T = (pre2 << 10) | (uint32_t)s_bin;  // the k-th largest key
+    krem = s_krem;                                       // keys equal to T to take
+
+    int gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        gt += key[e] > T;
+        eq += key[e] == T;
+    }
+    int total;
+    const int eq_before = block_excl_scan(eq, scan_buf, &total);
+    const int take_eq = max(0, min(eq, krem - eq_before));
+    int pos = block_excl_scan(gt + take_eq, scan_buf, &total);
+    int32_t* o = out + (int64_t)blockIdx.x * k;
+    int eq_seen = 0;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        bool take = key[e] > T;
+        if (key[e] == T) {
+            take = eq_seen < take_eq;
+            ++eq_seen;
+        }
+        if (take) {
+            if (pos < k) o[pos] = j0 + e;  // pos < k by construction; the bound keeps writes in the row
+            ++pos;
+        }
+    }
+}
+
+// Long rows: keys in shared memory (kSmem) or re-read from global memory,
+// 8-bit digits with warp-aggregated shared-memory atomics.
 template <bool kSmem>
-__global__ void __launch_bounds__(512) k_topk(const float* __restrict__ scores, int S, int k,
-                                              int32_t* __restrict__ out) {
+__global__ void __launch_bounds__(512) k_topk_long(const float* __restrict__ scores, int S, int k,
+                                                   int32_t* __restrict__ out) {
     extern __shared__ uint32_t keys[];
     __shared__ uint32_t hist[256];
-    __shared__ int s_digit, s_krem;
+    __shared__ int s_bin, s_krem;
     __shared__ int scan_buf[32];
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    if (tid == 0) {
-        s_digit = 0;
-        s_krem = k;
-    }
     const float* row = scores + (int64_t)blockIdx.x * S;
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (kSmem) {
         for (int j = tid; j < S; j += nt) keys[j] = order_key(__ldg(row + j));
@@ -85,36 +208,24 @@ __global__ void __launch_bounds__(512) k_topk(const float* __restrict__ scores, 
             if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
         }
         __syncthreads();
-        if (tid < 32) {
-            // lane l owns bins [8l, 8l + 8); higher bins hold larger keys
-            int c[8], tot = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                c[e] = (int)hist[8 * lane + e];
-                tot += c[e];
-            }
-            int suf = tot;  // inclusive suffix sum over lanes
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_down_sync(0xffffffffu, suf, off);
-                if (lane + off < 32) suf += y;
-            }
-            int above = suf - tot;
-#pragma unroll
-            for (int e = 7; e >= 0; --e) {
-                if (above < krem && above + c[e] >= krem) {
-                    s_digit = 8 * lane + e;
-                    s_krem = krem - above;
-                }
-                above += c[e];
+        // 256 bins over 512 threads: the first 256 threads own one bin each
+        {
+            const int c = tid < 256 ? (int)hist[tid] : 0;
+            int total;
+            const int before = block_excl_scan(c, scan_buf, &total);
+            const int above = total - before - c;
+            if (tid < 256 && above < krem && above + c >= krem) {
+                s_bin = tid;
+                s_krem = krem - above;
             }
         }
         __syncthreads();
-        prefix |= (uint32_t)s_digit << shift;
+        prefix |= (uint32_t)s_bin << shift;
         mask |= 0xffu << shift;
         krem = s_krem;
+        __syncthreads();
     }
-    const uint32_t T = prefix;  // the k-th largest key; take `krem` of the keys equal to T
+    const uint32_t T = prefix;
 
     const int per = (S + nt - 1) / nt;
     const int j0 = min(S, tid * per), j1 = min(S, j0 + per);
@@ -127,9 +238,8 @@ __global__ void __launch_bounds__(512) k_topk(const float* __restrict__ scores, 
     int total;
     const int eq_before = block_excl_scan(eq, scan_buf, &total);
     const int take_eq = max(0, min(eq, krem - eq_before));
-    const int off = block_excl_scan(gt + take_eq, scan_buf, &total);
+    int pos = block_excl_scan(gt + take_eq, scan_buf, &total);
     int32_t* o = out + (int64_t)blockIdx.x * k;
-    int pos = off;  // stays below k by construction; the bound keeps a row's writes in the row
     int eq_seen = 0;
     for (int j = j0; j < j1; ++j) {
         const uint32_t key = kSmem ? keys[j] : order_key(__ldg(row + j));
@@ -145,25 +255,37 @@ __global__ void __launch_bounds__(512) k_topk(const float* __restrict__ scores, 
     }
 }
 
+template <int KPT, int NT>
+static cudaError_t launch_reg(const float* scores, int64_t rows, int S, int k, int32_t* idx,
+                              cudaStream_t s, bool pdl) {
+    return launch_kernel(k_topk_reg<KPT, NT>, dim3((unsigned)rows), dim3(NT), 0, s, pdl, scores,
+                         S, k, idx);
+}
+
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
-                        cudaStream_t s) {
-    DevInfo di;
-    cudaError_t e = dev_info(&di);
-    if (e != cudaSuccess) return e;
-    const size_t static_smem = 256 * 4 + 32 * 4 + 16;
-    const size_t need = (size_t)S * 4;
-    const int threads = 512;
-    if (need + static_smem <= (size_t)di.smem_optin) {
-        if (need > 48 * 1024) {
-            e = cudaFuncSetAttribute(k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                        cudaStream_t s, bool pdl) {
+    const int Si = (int)S, ki = (int)k;
+    if (S <= 256 * 4) return launch_reg<4, 256>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 8) return launch_reg<8, 256>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 16) return launch_reg<16, 256>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 512 * 16) return launch_reg<16, 512>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 512 * 32) return launch_reg<32, 512>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 512 * 64) return launch_reg<64, 512>(scores, rows, Si, ki, idx, s, pdl);
+    {
+        DevInfo di;
+        cudaError_t e = dev_info(&di);
+        if (e != cudaSuccess) return e;
+        const size_t need = (size_t)S * 4;
+        if (need + 4096 <= (size_t)di.smem_optin) {
+            e = cudaFuncSetAttribute(k_topk_long<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)need);
             if (e != cudaSuccess) return e;
+            return launch_kernel(k_topk_long<true>, dim3((unsigned)rows), dim3(512), need, s, pdl,
+                                 scores, Si, ki, idx);
         }
-        k_topk<true><<<(unsigned)rows, threads, need, s>>>(scores, (int)S, (int)k, idx);
-    } else {
-        k_topk<false><<<(unsigned)rows, threads, 0, s>>>(scores, (int)S, (int)k, idx);
+        return launch_kernel(k_topk_long<false>, dim3((unsigned)rows), dim3(512), 0, s, pdl,
+                             scores, Si, ki, idx);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace loki

@@ -111,6 +111,31 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert lib.loki_project_query(FAKE, FAKE, 1, 1, 1, 128, L.DTYPE_F32, FAKE + 4, None) == 1
 
 
+def test_plane_entry_points_reject_bad_arguments(L):
+    lib = L.lib
+    ws = lib.loki_decode_workspace_size(1, 2, 2, 100, 128, 32, 10)
+
+    def args(**kw):
+        return dict(dict(Kt_lo=FAKE, d_lo=32, d=32), **kw)
+
+    def dec(Kt_lo, d_lo, d):
+        return lib.loki_decode_attention_plane(FAKE, FAKE, FAKE, Kt_lo, d_lo, FAKE, 1, 2, 2, 100,
+                                               100, 128, d, 10, 0.0, L.DTYPE_BF16, FAKE, FAKE,
+                                               FAKE, ws, None)
+    assert dec(**args(d=33)) == 1            # d > d_lo
+    assert dec(**args(d_lo=20, d=16)) == 1   # d_lo * 2 bytes not a multiple of 16
+    assert dec(**args(Kt_lo=None)) == 1
+    assert dec(**args(Kt_lo=FAKE + 8)) == 1  # misaligned plane
+    assert lib.loki_append_keys_plane(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 129, 1, 2, 1, 128, 10,
+                                      0, L.DTYPE_BF16, None) == 1
+    # the score scan takes a plane's row width: rows must be a multiple of 16 bytes
+    # (20 bf16 = 40 bytes is not) and hold at least d columns
+    assert lib.loki_score_lowdim(FAKE, FAKE, 1, 1, 1, 10, 10, 20, 8, L.DTYPE_BF16, FAKE,
+                                 None) == 1
+    assert lib.loki_score_lowdim(FAKE, FAKE, 1, 1, 1, 10, 10, 24, 25, L.DTYPE_BF16, FAKE,
+                                 None) == 1
+
+
 def test_python_binding_requires_cuda_tensors():
     torch = pytest.importorskip("torch")
     import sparse_attention_decode_loki_b200 as loki

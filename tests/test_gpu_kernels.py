@@ -166,6 +166,32 @@ def test_append_matches_oracle_rotation(loki, cuda, dtype, T, pos):
     assert np.abs(back - inp.K).max() < (0.05 if dtype == "bf16" else 1e-4)
 
 
+@pytest.mark.parametrize("dtype,d_lo", [("bf16", 32), ("bf16", 16), ("f32", 36)])
+def test_append_plane_copies_the_low_columns(loki, cuda, dtype, d_lo):
+    torch = _t()
+    wl = workloads.get("llama2-7b").with_(B=2, H_q=3, H_kv=3, S=9, dtype=dtype, n_cal=512,
+                                          name=f"append-plane-{dtype}")
+    inp = parity.host_inputs(wl)
+    dt = parity.torch_dtype(wl)
+    S_max, pos = 40, 17
+    Kc = torch.zeros((2, 3, S_max, 128), dtype=dt, device=cuda)
+    Vc = torch.zeros_like(Kc)
+    Klo = torch.full((2, 3, S_max, d_lo), 9.0, dtype=dt, device=cuda)
+    K2 = torch.zeros_like(Kc)
+    V2 = torch.zeros_like(Kc)
+    P = torch.from_numpy(inp.P).to(cuda)
+    Kn, Vn = parity.to_device(inp.K, wl, cuda), parity.to_device(inp.V, wl, cuda)
+    loki.loki_append_keys(Kn, Vn, P, Kc, Vc, pos, Kt_lo=Klo)
+    loki.loki_append_keys(Kn, Vn, P, K2, V2, pos)
+    # the rotated rows are the same with or without the plane, and the plane
+    # holds exactly their first d_lo columns; other plane rows are untouched
+    assert torch.equal(Kc, K2) and torch.equal(Vc, V2)
+    assert torch.equal(Klo[:, :, pos:pos + wl.S], Kc[:, :, pos:pos + wl.S, :d_lo])
+    mask = torch.ones(S_max, dtype=torch.bool)
+    mask[pos:pos + wl.S] = False
+    assert bool((Klo[:, :, mask] == 9.0).all())
+
+
 # ---------------------------------------------------------------------------
 # calibration: eigenvalues, vectors where the spectrum separates them,
 # subspaces at every d used by the workloads

@@ -27,7 +27,7 @@ def _torch():
     return torch
 
 
-def run_full(loki, inp, dev, S=None, S_max=None, d=None, k=None, with_steps=False):
+def run_full(loki, inp, dev, S=None, S_max=None, d=None, k=None, with_steps=False, d_lo=None):
     torch = _torch()
     wl = inp.wl
     S = wl.S if S is None else S
@@ -37,12 +37,17 @@ def run_full(loki, inp, dev, S=None, S_max=None, d=None, k=None, with_steps=Fals
     Kt = parity.to_device(inp.Kt[:, :, :S], wl, dev, S_max=S_max)
     V = parity.to_device(inp.V[:, :, :S], wl, dev, S_max=S_max)
     P = torch.from_numpy(inp.P).to(dev)
-    out, idx = loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale)
+    Kt_lo = None
+    if d_lo is not None:
+        # the low-dim key plane holds a copy of the first d_lo rotated columns
+        Kt_lo = parity.to_device(inp.Kt[:, :, :S, :d_lo], wl, dev, S_max=S_max)
+    out, idx = loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, Kt_lo=Kt_lo)
     res = {"out": out.float().cpu().numpy(), "idx": idx.cpu().numpy()}
     if with_steps:
         q_rot = loki.loki_project_query(q, P)
         res["q_rot"] = q_rot.cpu().numpy()
-        res["scores"] = loki.loki_score_lowdim(q_rot, Kt, S, d).cpu().numpy()
+        res["scores"] = loki.loki_score_lowdim(q_rot, Kt if Kt_lo is None else Kt_lo, S,
+                                               d).cpu().numpy()
     torch.cuda.synchronize()
     return res
 
@@ -107,6 +112,28 @@ def test_edge_cases(loki, cuda, dtype, name, over, S_max):
     check_all_rows(inp, res, steps=True)
 
 
+@pytest.mark.parametrize("name,d_lo", [("tiny", 32), ("tiny", 36), ("llama2-7b", 32),
+                                       ("llama2-7b", 64)])
+def test_plane_layout_full(loki, cuda, name, d_lo):
+    inp = parity.host_inputs(workloads.get(name))
+    res = run_full(loki, inp, cuda, S_max=inp.wl.S + 64, with_steps=True, d_lo=d_lo)
+    check_all_rows(inp, res, steps=True)
+
+
+PLANE_EDGE = [("ragged-S-d20", 24), ("d1", 8), ("d-full", 128), ("gqa4", 16), ("gqa3", 40),
+              ("k1", 32)]
+
+
+@pytest.mark.parametrize("name,d_lo", PLANE_EDGE, ids=[e[0] for e in PLANE_EDGE])
+def test_plane_edge_cases(loki, cuda, name, d_lo):
+    over, S_max = {e[0]: (e[1], e[2]) for e in EDGE}[name]
+    wl = workloads.get("llama2-7b").with_(B=1, H_q=2, H_kv=2, n_cal=512,
+                                          name=f"edge-{name}-bf16").with_(**over)
+    inp = parity.host_inputs(wl)
+    res = run_full(loki, inp, cuda, S_max=S_max, with_steps=True, d_lo=d_lo)
+    check_all_rows(inp, res, steps=True)
+
+
 def test_all_dims_all_tokens_is_dense(loki, cuda):
     torch = _torch()
     wl = workloads.get("llama2-7b").with_(H_q=4, H_kv=4, S=1024, name="dense-invariant")
@@ -132,7 +159,7 @@ def test_all_dims_all_tokens_is_dense(loki, cuda):
 # large workloads: full launch, sampled rows
 # ---------------------------------------------------------------------------
 
-def sampled_run(loki, dev, wl, n_rows, seed=7):
+def sampled_run(loki, dev, wl, n_rows, seed=7, plane=False):
     """Full-size launch; the sampled rows' blocks hold generator + oracle bytes,
     every other block holds seeded random filler (its rows are not checked)."""
     torch = _torch()
@@ -161,7 +188,8 @@ def sampled_run(loki, dev, wl, n_rows, seed=7):
             V[b, hk] = torch.from_numpy(Vb).to(dev).to(dt)
         q[b, h] = torch.from_numpy(workloads.query_vec(wl, b, h, Rs[hk])).to(dev).to(dt)
     Pt = torch.from_numpy(P).to(dev)
-    out, idx = loki.loki_decode_attention(q, Kt, V, Pt, wl.S, wl.d, wl.k, wl.scale)
+    Kt_lo = Kt[..., : wl.d].contiguous() if plane else None
+    out, idx = loki.loki_decode_attention(q, Kt, V, Pt, wl.S, wl.d, wl.k, wl.scale, Kt_lo=Kt_lo)
     out = out.float().cpu().numpy()
     idx = idx.cpu().numpy()
     qh = q.float().cpu().numpy()
@@ -182,13 +210,15 @@ def _check_block(wl, P, q, Kt, V, gidx, gout, row):
     return parity.check_row(inp, 0, 0, gidx, gout, wl.d, wl.k, wl.scale)
 
 
-def test_llama2_13b_sampled(loki, cuda):
-    s = sampled_run(loki, cuda, workloads.get("llama2-13b"), 24)
+@pytest.mark.parametrize("plane", [False, True])
+def test_llama2_13b_sampled(loki, cuda, plane):
+    s = sampled_run(loki, cuda, workloads.get("llama2-13b"), 24, plane=plane)
     assert s["rows"] == 24
 
 
-def test_llama3_8b_gqa_sampled(loki, cuda):
-    s = sampled_run(loki, cuda, workloads.get("llama3-8b-gqa"), 16)
+@pytest.mark.parametrize("plane", [False, True])
+def test_llama3_8b_gqa_sampled(loki, cuda, plane):
+    s = sampled_run(loki, cuda, workloads.get("llama3-8b-gqa"), 16, plane=plane)
     assert s["rows"] == 16
 
 
@@ -199,7 +229,7 @@ SWEEP_SAMPLE = ["sweep-B1-S2048-d16-k1of8", "sweep-B8-S16384-d32-k1of4",
 
 @pytest.mark.parametrize("name", SWEEP_SAMPLE)
 def test_sweep_sampled(loki, cuda, name):
-    s = sampled_run(loki, cuda, workloads.get(name), 6)
+    s = sampled_run(loki, cuda, workloads.get(name), 6, plane=True)
     assert s["rows"] == 6
 
 
