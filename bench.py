@@ -40,7 +40,7 @@ METRIC = "Loki decode-attn µs/layer-step, HBM GB/s (% roofline), speedup vs den
 UNIT = "us/layer-step"
 FALLBACK_HBM_GBS = 6650.0
 LAUNCHES_PER_DECODE = 5  # project, score, top-k, sparse attention, combine
-L2_FLUSH_BYTES = 256 << 20
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB of L2
 
 
 def parse_args():
@@ -280,8 +280,22 @@ def run_ours(args):
     idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
     ws = torch.empty(loki.loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k),
                      dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    class _Flush:
+        """Evict L2 before a timed step: write 256 MiB (the write-flush), then read
+        another 256 MiB so the dirty lines are written back here, outside the timed
+        region, and the step starts with a cold, clean L2."""
+
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.sum(flush_r, out=flush_sink)
+
+    flush = _Flush()
 
     def decode():
         loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
@@ -305,15 +319,29 @@ def run_ours(args):
         torch.cuda.synchronize()
         return [s.elapsed_time(t) for s, t in zip(starts, ends)]
 
+    # One decode call is captured once into a CUDA graph: the replay launches
+    # exactly the kernels the call launches (same C-ABI call, same arguments),
+    # without the Python/ctypes issue time between them.
+    decode()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            decode()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+
     # ---- the timed region: exactly K decode steps --------------------------------
     for _ in range(args.warmup):
         flush.zero_()
-        decode()
+        graph.replay()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        step_ms = timed(decode, args.steps, 0)
+        step_ms = timed(graph.replay, args.steps, 0)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -324,33 +352,29 @@ def run_ours(args):
         total_ms = float(t.item())
     us_per_step_rank = total_ms * 1e3 / args.steps
     value = us_per_step_rank / world
+    nb = max(50, min(args.steps, 400))
+    eager_us = statistics.mean(timed(decode, nb, 10)) * 1e3
 
-    # ---- per-kernel breakdown through the step entry points ----------------------
+    # ---- per-kernel times: each step entry point alone, after an L2 flush -------
     q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
     scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
     sp_ws = torch.empty(loki.loki_sparse_attention_workspace_size(B, H_q, k, D), dtype=torch.uint8,
                         device=dev)
-    nb = max(50, min(args.steps, 400))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nb)]
-    for i in range(nb + 10):
-        flush.zero_()
-        ev = evs[i - 10] if i >= 10 else None
-        if ev: ev[0].record(stream)
-        loki.loki_project_query(q, P, q_rot)
-        if ev: ev[1].record(stream)
-        loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores)
-        if ev: ev[2].record(stream)
-        loki.loki_topk(scores, k, idx)
-        if ev: ev[3].record(stream)
-        loki.loki_sparse_attention(q_rot, Kt, V, idx, S, wl.scale, out, sp_ws)
-        if ev: ev[4].record(stream)
-    torch.cuda.synchronize()
-    names = ["project_query", "score_lowdim", "topk", "sparse_attention+combine"]
-    kern_us = {n: statistics.mean(e_[j].elapsed_time(e_[j + 1]) for e_ in evs) * 1e3
-               for j, n in enumerate(names)}
+    loki.loki_project_query(q, P, q_rot)
+    loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores)
+    loki.loki_topk(scores, k, idx)
+    comps = {
+        "project_query": lambda: loki.loki_project_query(q, P, q_rot),
+        "score_lowdim": lambda: loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores),
+        "topk": lambda: loki.loki_topk(scores, k, idx),
+        "sparse_attention+combine": lambda: loki.loki_sparse_attention(q_rot, Kt, V, idx, S,
+                                                                       wl.scale, out, sp_ws),
+    }
+    kern_us = {n_: statistics.mean(timed(f_, nb, 10)) * 1e3 for n_, f_ in comps.items()}
 
     # ---- the same step on the row-only cache layout (no low-dim plane) ---------
     rows_only_us = statistics.mean(timed(decode_rows_only, nb, 10)) * 1e3
+    del graph
 
     # ---- dense baseline on the same cache (q~ rounded to the cache dtype) ------
     q_rot_dt = loki.loki_project_query(q, P).to(q.dtype)
@@ -417,12 +441,16 @@ def run_ours(args):
         "config": {"workload": wl.name, "B": B, "H_q": H_q, "H_kv": H_kv, "D": D, "S": S,
                    "d": d, "k": k, "cache_dtype": wl.dtype,
                    "cache_layout": "rotated K rows + contiguous d-column key plane",
-                   "l2": "flushed (256 MiB write) before every timed step, flush excluded",
+                   "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read "
+                         "so no dirty lines remain), flush excluded from the timing",
+                   "timing": "CUDA-graph replay of one loki_decode_attention_plane call per step, "
+                             "CUDA events on the launching stream",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "tokens_per_s": round(B * world * 1e6 / us_per_step_rank, 1),
         "hbm_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
         "hbm_frac_of_" + peak_kind: round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 4),
-        "rows_only_layout_us": round(rows_only_us, 3),
+        "eager_us": round(eager_us, 3),
+        "rows_only_layout_eager_us": round(rows_only_us, 3),
         "dense_us": round(dense_us, 3),
         "speedup_vs_dense": round(dense_us / step_us, 3),
         "append_us": round(append_us, 3),
@@ -505,9 +533,13 @@ def run_ncu_case(args):
     Kt = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
     V = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
     q = torch.randn((wl.B, wl.H_q, wl.D), generator=g, device=dev, dtype=dt)
-    P = torch.linalg.qr(torch.randn((wl.H_kv, wl.D, wl.D), generator=g, device=dev))[0].contiguous()
+    Kt_lo = Kt[..., : wl.d].contiguous()
+    # an orthonormal basis from the host (seeded), so the launch list holds only this library
+    import numpy as np
+    Pn = np.linalg.qr(np.random.default_rng(wl.seed).standard_normal((wl.H_kv, wl.D, wl.D)))[0]
+    P = torch.from_numpy(np.ascontiguousarray(Pn, dtype=np.float32)).to(dev)
     for _ in range(max(1, args.steps)):
-        loki.loki_decode_attention(q, Kt, V, P, wl.S, wl.d, wl.k, wl.scale)
+        loki.loki_decode_attention(q, Kt, V, P, wl.S, wl.d, wl.k, wl.scale, Kt_lo=Kt_lo)
     for _ in range(2):
         loki.dense_decode_attention(q, Kt, V, wl.S, wl.scale)
     Kc = torch.empty((wl.B, wl.H_kv, 8, wl.D), dtype=dt, device=dev)

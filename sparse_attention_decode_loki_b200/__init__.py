@@ -50,6 +50,11 @@ def _cuda(*ts: torch.Tensor) -> torch.device:
     return dev
 
 
+def _expect(t: torch.Tensor, shape, dtype, name: str) -> None:
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {list(shape)} (got {t.dtype} {list(t.shape)})")
+
+
 def _stream(dev: torch.device) -> int:
     return torch.cuda.current_stream(dev).cuda_stream
 
@@ -103,6 +108,8 @@ def loki_calibrate_pca(keys: torch.Tensor, P: Optional[torch.Tensor] = None,
     if eigvals is None:
         eigvals = torch.empty((H_kv, D), dtype=torch.float32, device=dev)
     _cuda(keys, P, eigvals)
+    _expect(P, (H_kv, D, D), torch.float32, "P")
+    _expect(eigvals, (H_kv, D), torch.float32, "eigvals")
     ws = _ws(loki_calibrate_workspace_size(N, H_kv, D), dev, workspace)
     check(lib.loki_calibrate_pca(keys.data_ptr(), _dt(keys), N, H_kv, D, P.data_ptr(),
                                  eigvals.data_ptr(), ws.data_ptr(), _ws_bytes(ws), _stream(dev)),
@@ -149,6 +156,7 @@ def loki_append_keys_plane(K_new, V_new, P, Kt_cache, V_cache, Kt_lo, pos: int) 
 
 def _check_plane(Kt_lo: torch.Tensor, Kt_cache: torch.Tensor) -> None:
     _cuda(Kt_lo, Kt_cache)
+    # the C library takes d_lo from Kt_lo.shape[3] and strides the plane by it
     if Kt_lo.dim() != 4 or Kt_lo.shape[:3] != Kt_cache.shape[:3] or Kt_lo.dtype != Kt_cache.dtype:
         raise ValueError("Kt_lo must be [B, H_kv, S_max, d_lo] with the cache's dtype")
 
@@ -184,6 +192,10 @@ def loki_decode_attention(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torc
     if selected_idx is None:
         selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
     _cuda(q, out, selected_idx)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    if S > S_max:
+        raise ValueError("S must be <= S_max")
     ws = _ws(loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k), dev, workspace)
     if Kt_lo is None:
         check(lib.loki_decode_attention(q.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
@@ -216,8 +228,11 @@ def loki_project_query(q: torch.Tensor, P: torch.Tensor,
     dev = _cuda(q, P)
     B, H_q, D = q.shape
     H_kv = P.shape[0]
+    _expect(P, (H_kv, D, D), torch.float32, "P")
     if q_rot is None:
         q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
+    _cuda(q, q_rot)
+    _expect(q_rot, (B, H_q, D), torch.float32, "q_rot")
     check(lib.loki_project_query(q.data_ptr(), P.data_ptr(), B, H_q, H_kv, D, _dt(q),
                                  q_rot.data_ptr(), _stream(dev)), "loki_project_query")
     return q_rot
@@ -225,15 +240,25 @@ def loki_project_query(q: torch.Tensor, P: torch.Tensor,
 
 def loki_score_lowdim(q_rot: torch.Tensor, Kt_cache: torch.Tensor, S: int, d: int,
                       scores: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """fp32 scores [B, H_q, S] on the first d rotated dimensions."""
+    """fp32 scores [B, H_q, S] on the first d rotated dimensions.
+
+    Kt_cache is the rotated cache [B, H_kv, S_max, 128] or a low-dimensional
+    key plane [B, H_kv, S_max, d_lo]; its last dimension is the row width the
+    scan strides by.
+    """
     dev = _cuda(q_rot, Kt_cache)
-    B, H_q, D = q_rot.shape
-    _, H_kv, S_max, _ = Kt_cache.shape
-    if q_rot.dtype != torch.float32:
-        raise TypeError("q_rot must be float32")
+    B, H_q, Dq = q_rot.shape
+    Bk, H_kv, S_max, row = Kt_cache.shape
+    if q_rot.dtype != torch.float32 or Dq != 128:
+        raise TypeError("q_rot must be float32 [B, H_q, 128]")
+    if Bk != B or not 1 <= d <= row or S > S_max:
+        raise ValueError("Kt_cache must be [B, H_kv, S_max >= S, row >= d]")
     if scores is None:
         scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
-    check(lib.loki_score_lowdim(q_rot.data_ptr(), Kt_cache.data_ptr(), B, H_q, H_kv, S, S_max, D,
+    if scores.shape != (B, H_q, S) or scores.dtype != torch.float32:
+        raise ValueError("scores must be float32 [B, H_q, S]")
+    _cuda(q_rot, scores)
+    check(lib.loki_score_lowdim(q_rot.data_ptr(), Kt_cache.data_ptr(), B, H_q, H_kv, S, S_max, row,
                                 d, _dt(Kt_cache), scores.data_ptr(), _stream(dev)),
           "loki_score_lowdim")
     return scores
@@ -248,6 +273,8 @@ def loki_topk(scores: torch.Tensor, k: int, selected_idx: Optional[torch.Tensor]
     rows = scores.numel() // S
     if selected_idx is None:
         selected_idx = torch.empty((*scores.shape[:-1], k), dtype=torch.int32, device=dev)
+    _cuda(scores, selected_idx)
+    _expect(selected_idx, (*scores.shape[:-1], k), torch.int32, "selected_idx")
     ws = _ws(loki_topk_workspace_size(rows, S, k), dev, None)
     check(lib.loki_topk(scores.data_ptr(), rows, S, k, selected_idx.data_ptr(), ws.data_ptr(),
                         _ws_bytes(ws), _stream(dev)), "loki_topk")
@@ -261,12 +288,17 @@ def loki_sparse_attention(q_rot: torch.Tensor, Kt_cache: torch.Tensor, V_cache: 
     """Exact attention of q~ over the selected tokens; out has the caches' dtype."""
     dev = _cuda(q_rot, Kt_cache, V_cache, selected_idx)
     B, H_q, D = q_rot.shape
-    _, H_kv, S_max, _ = Kt_cache.shape
+    Bk, H_kv, S_max, Dk = Kt_cache.shape
     k = selected_idx.shape[-1]
-    if selected_idx.dtype != torch.int32:
-        raise TypeError("selected_idx must be int32")
+    _expect(q_rot, (B, H_q, D), torch.float32, "q_rot")
+    _expect(V_cache, Kt_cache.shape, Kt_cache.dtype, "V_cache")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    if Bk != B or Dk != D or S > S_max:
+        raise ValueError("Kt_cache must be [B, H_kv, S_max >= S, D]")
     if out is None:
         out = torch.empty((B, H_q, D), dtype=Kt_cache.dtype, device=dev)
+    _cuda(q_rot, out)
+    _expect(out, (B, H_q, D), Kt_cache.dtype, "out")
     ws = _ws(loki_sparse_attention_workspace_size(B, H_q, k, D), dev, workspace)
     check(lib.loki_sparse_attention(q_rot.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
                                     selected_idx.data_ptr(), B, H_q, H_kv, S, S_max, D, k,
@@ -282,6 +314,10 @@ def dense_decode_attention(q: torch.Tensor, K_cache: torch.Tensor, V_cache: torc
     dev, B, H_q, H_kv, S_max, D = _check_decode(q, K_cache, V_cache)
     if out is None:
         out = torch.empty_like(q)
+    _cuda(q, out)
+    _expect(out, q.shape, q.dtype, "out")
+    if S > S_max:
+        raise ValueError("S must be <= S_max")
     ws = _ws(dense_decode_workspace_size(B, H_q, H_kv, S, D), dev, workspace)
     check(lib.dense_decode_attention(q.data_ptr(), K_cache.data_ptr(), V_cache.data_ptr(), B, H_q,
                                      H_kv, S, S_max, D, float(scale), _dt(q), out.data_ptr(),

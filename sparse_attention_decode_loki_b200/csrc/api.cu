@@ -108,7 +108,7 @@ struct DecodeWs {
 };
 DecodeWs decode_ws(int B, int H_q, int64_t S, int D, int64_t k) {
     const int64_t rows = (int64_t)B * H_q;
-    const int64_t parts = loki::sparse_max_parts(k);
+    const int64_t parts = loki::sparse_max_parts(rows, k);
     DecodeWs w;
     w.q_rot = 0;
     w.scores = align_up(w.q_rot + (size_t)rows * D * sizeof(float));
@@ -123,7 +123,7 @@ struct SparseWs {
 };
 SparseWs sparse_ws(int B, int H_q, int64_t k, int D) {
     const int64_t rows = (int64_t)B * H_q;
-    const int64_t parts = loki::sparse_max_parts(k);
+    const int64_t parts = loki::sparse_max_parts(rows, k);
     SparseWs w;
     w.ml = 0;
     w.acc = align_up((size_t)rows * parts * sizeof(float2));

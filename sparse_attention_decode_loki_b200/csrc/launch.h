@@ -34,8 +34,8 @@ cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl);
 
-// split-k partial slots per (batch, query head) row
-int64_t sparse_max_parts(int64_t k);
+// partial slots per (batch, query head) row of the sparse attention split
+int64_t sparse_max_parts(int64_t rows, int64_t k);
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,

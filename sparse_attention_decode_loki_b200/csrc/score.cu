@@ -36,16 +36,42 @@ __global__ void __launch_bounds__(256) k_project_query(const typename E::T* __re
     const int nrows = min(kProjRows, B * G - r0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float* Ph = P + (int64_t)hk * D * D;
-    for (int it = tid; it < D * kProjCols; it += 256) {
-        const int i = it / kProjCols, c = it % kProjCols;
-        Ps[i][c] = (c0 + c < D) ? __ldg(Ph + (int64_t)i * D + c0 + c) : 0.f;
+    // P block: 128 rows x 32 columns = 1024 float4, 4 per thread, all in flight
+    float4 pv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int it = tid + u * 256;
+        const int i = it >> 3, c4 = (it & 7) * 4;
+        pv[u] = (i < D && c0 + c4 < D)
+                    ? __ldg(reinterpret_cast<const float4*>(Ph + (int64_t)i * D + c0 + c4))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    // the head's queries: row j of the chunk is (batch b, group member g)
-    for (int it = tid; it < nrows * D; it += 256) {
+    // the head's queries: row j of the chunk is (batch b, group member g);
+    // 8 consecutive elements per thread per step
+    constexpr int QV = 8;
+    float qv[kProjRows * 128 / 256];
+#pragma unroll
+    for (int u = 0; u < kProjRows * 128 / 256 / QV; ++u) {
+        const int it = (tid + u * 256) * QV;
         const int j = it / D, i = it % D;
         const int jr = r0 + j;
         const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
-        qs[j][i] = E::load1(q + row * D + i);
+#pragma unroll
+        for (int e = 0; e < QV; ++e)
+            qv[u * QV + e] = (j < nrows) ? E::load1(q + row * D + i + e) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int it = tid + u * 256;
+        const int i = it >> 3, c4 = (it & 7) * 4;
+        if (i < 128) *reinterpret_cast<float4*>(&Ps[i][c4]) = pv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kProjRows * 128 / 256 / QV; ++u) {
+        const int it = (tid + u * 256) * QV;
+        const int j = it / D, i = it % D;
+#pragma unroll
+        for (int e = 0; e < QV; ++e) qs[j][i + e] = qv[u * QV + e];
     }
     __syncthreads();
     for (int j = warp; j < nrows; j += 8) {

@@ -3,58 +3,60 @@
 // "Visual Insights" Figure 1 caption: the full-dimensional keys give the
 // final attention scores).
 //
-// Work items are (row, j) pairs, row = (batch, query head) and j < k the
-// position in its selected list; the B*H_q*k items are split evenly over one
-// wave of CTAs. Each CTA stages its selected indices in shared memory (1024
-// at a time), so the row gathers never wait on an index load. A row group of
-// lanes (16 lanes for bf16, 32 for fp32) owns one 256/512-byte key row and
-// the matching value row per step, with 8 rows in flight; each row is a
-// random gather, but a contiguous one. Scores use all D
-// dimensions in fp32; the softmax runs online in base 2 with the scale folded
-// into q~. Each CTA merges its row groups and writes one partial per row
-// segment; k_combine merges the partials of a row.
-#include "combine.cuh"
+// One warp per (row, chunk of the selected list); no block barriers. The warp
+// stages its selected indices in shared memory, then each row group of lanes
+// (16 lanes for bf16, 32 for fp32) gathers one 256/512-byte key row and the
+// matching value row per step, 8 rows in flight; every row is a random but
+// contiguous gather. Scores use all D dimensions in fp32; the softmax runs
+// online in base 2 with the scale folded into q~. The warp merges its row
+// groups with shuffles and writes one partial; k_combine_rows merges a row's
+// partials.
 #include "common.cuh"
 #include "launch.h"
 
 namespace loki {
 
-constexpr int kSparseMinItems = 64;  // CTAs own at least this many items
+// Work decomposition. Each (batch, query head) row's k selected positions are
+// cut into nchunk chunks; a work item is one (row, chunk) and one warp owns one
+// item at a time (grid-stride over items). nchunk is chosen so the items fill
+// one wave of resident warps. Partials of row r sit in slots [r*nchunk, ...).
+constexpr int kMinChunk = 16;
+constexpr int kWarpIdx = 256;  // indices staged per warp per step
 
-// A CTA of the split owns per >= kSparseMinItems / 2 items (grid <= total /
-// kSparseMinItems, rounded up), so a row of k items spans at most
-// (k - 1) / per + 2 CTAs; the workspace is sized for the smallest per.
-int64_t sparse_max_parts(int64_t k) { return (k - 1) / (kSparseMinItems / 2) + 2; }
+int64_t sparse_max_parts(int64_t rows, int64_t k) {
+    int64_t cap = 10240 / rows;
+    if (cap < 1) cap = 1;
+    const int64_t by_k = (k + kMinChunk - 1) / kMinChunk;
+    return by_k < cap ? by_k : cap;
+}
 
 template <class E>
-__global__ void __launch_bounds__(256, 2) k_sparse_attn(
+__global__ void __launch_bounds__(256) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
-    int64_t S_max, int k, float scale_log2, int64_t total, int64_t per, int maxp,
+    int64_t S_max, int k, float scale_log2, int chunk, int nchunk, int64_t n_items,
     float2* __restrict__ part_ml, float* __restrict__ part_acc) {
     constexpr int D = 128;
     constexpr int KV = E::kVec;
-    constexpr int LPR = D / KV;           // lanes per row
-    constexpr int NGRP = 256 / LPR;       // row groups per CTA
-    constexpr int U = 8;                  // rows in flight per group
-    constexpr int kIdxChunk = 1024;       // selected indices staged per step
+    constexpr int LPR = D / KV;     // lanes per row
+    constexpr int GPW = 32 / LPR;   // row groups per warp
+    constexpr int U = 8;            // rows in flight per group
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
-    __shared__ float sm_m[NGRP], sm_l[NGRP];
-    __shared__ float sm_acc[NGRP][D];
-    __shared__ int s_idx[kIdxChunk];
+    __shared__ int s_idx[8][kWarpIdx];
 
-    const int grp = threadIdx.x / LPR;
-    const int sub = threadIdx.x % LPR;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int grp = lane / LPR, sub = lane % LPR;
     const int G = H_q / H_kv;
+    int* widx = s_idx[warp];
     griddep_wait();  // q_rot and the selected indices come from earlier kernels
     griddep_launch_dependents();
 
-    int64_t w = (int64_t)blockIdx.x * per;
-    const int64_t w_end = min64(w + per, total);
-    while (w < w_end) {
-        const int64_t r = w / k;
-        const int j0 = (int)(w - r * k);
-        const int j1 = (int)min64(k, j0 + (w_end - w));
+    const int64_t nwarps = (int64_t)gridDim.x * 8;
+    for (int64_t item = (int64_t)blockIdx.x * 8 + warp; item < n_items; item += nwarps) {
+        const int64_t r = item / nchunk;
+        const int c = (int)(item - r * nchunk);
+        const int j0 = c * chunk;
+        const int j1 = min(k, j0 + chunk);
         const int b = (int)(r / H_q), h = (int)(r % H_q);
         const int64_t unit = (int64_t)b * H_kv + h / G;
 
@@ -72,21 +74,21 @@ __global__ void __launch_bounds__(256, 2) k_sparse_attn(
 #pragma unroll
         for (int e = 0; e < KV; ++e) acc[e] = 0.f;
 
-        for (int cb = j0; cb < j1; cb += kIdxChunk) {
-            const int n = min(kIdxChunk, j1 - cb);
-            __syncthreads();  // the previous chunk's indices are no longer read
-            for (int t = threadIdx.x; t < n; t += 256) {
+        for (int cb = j0; cb < j1; cb += kWarpIdx) {
+            const int n = min(kWarpIdx, j1 - cb);
+            __syncwarp();
+            for (int t = lane; t < n; t += 32) {
                 const int tok = __ldg(ip + cb + t);
-                s_idx[t] = ((unsigned)tok < (unsigned)S) ? tok : -1;
+                widx[t] = ((unsigned)tok < (unsigned)S) ? tok : -1;
             }
-            __syncthreads();
-            for (int jb = 0; jb < n; jb += NGRP * U) {
+            __syncwarp();
+            for (int jb = 0; jb < n; jb += GPW * U) {
                 int t[U];
                 uint4 kv[U], vv[U];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int jj = jb + u * NGRP + grp;
-                    const int tok = jj < n ? s_idx[jj] : -1;
+                    const int jj = jb + u * GPW + grp;
+                    const int tok = jj < n ? widx[jj] : -1;
                     t[u] = tok;
                     if (tok >= 0) {
                         kv[u] = ld_stream(Kb + (int64_t)tok * kRowBytes);
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(256, 2) k_sparse_attn(
                         vv[u] = kv[u];
                     }
                 }
-                float s[U];
+                float sc[U];
                 float mx = m;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -106,8 +108,8 @@ __global__ void __launch_bounds__(256, 2) k_sparse_attn(
 #pragma unroll
                     for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
                     a = group_sum<LPR>(a);
-                    s[u] = t[u] >= 0 ? a : -INFINITY;
-                    mx = fmaxf(mx, s[u]);
+                    sc[u] = t[u] >= 0 ? a : -INFINITY;
+                    mx = fmaxf(mx, sc[u]);
                 }
                 if (mx == -INFINITY) continue;
                 const float alpha = exp2f(m - mx);
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(256, 2) k_sparse_attn(
                 for (int e = 0; e < KV; ++e) acc[e] *= alpha;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const float p = exp2f(s[u] - mx);
+                    const float p = exp2f(sc[u] - mx);
                     l += p;
                     float f[KV];
                     E::unpack(vv[u], f);
@@ -126,35 +128,54 @@ __global__ void __launch_bounds__(256, 2) k_sparse_attn(
                 m = mx;
             }
         }
-
-        if (sub == 0) {
-            sm_m[grp] = m;
-            sm_l[grp] = l;
-        }
+        // merge the warp's row groups (lane l and lane l + LPR hold the same columns)
 #pragma unroll
-        for (int e = 0; e < KV; ++e) sm_acc[grp][sub * KV + e] = acc[e];
-        __syncthreads();
-        if (threadIdx.x < D) {
-            float M = -INFINITY;
+        for (int off = LPR; off < 32; off <<= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+            const float lo = __shfl_xor_sync(0xffffffffu, l, off);
+            const float M = fmaxf(m, mo);
+            const float sa = M == -INFINITY ? 0.f : exp2f(m - M);
+            const float sb = M == -INFINITY ? 0.f : exp2f(mo - M);
+            l = l * sa + lo * sb;
 #pragma unroll
-            for (int g = 0; g < NGRP; ++g) M = fmaxf(M, sm_m[g]);
-            float Lsum = 0.f, A = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int g = 0; g < NGRP; ++g) {
-                    const float sc = exp2f(sm_m[g] - M);
-                    Lsum += sm_l[g] * sc;
-                    A += sm_acc[g][threadIdx.x] * sc;
-                }
+            for (int e = 0; e < KV; ++e) {
+                const float ao = __shfl_xor_sync(0xffffffffu, acc[e], off);
+                acc[e] = acc[e] * sa + ao * sb;
             }
-            const int part = (int)(blockIdx.x - (r * k) / per);
-            const int64_t slot = r * maxp + part;
-            part_acc[slot * D + threadIdx.x] = A;
-            if (threadIdx.x == 0) part_ml[slot] = make_float2(M, Lsum);
+            m = M;
         }
-        __syncthreads();
-        w += j1 - j0;
+        if (grp == 0) {
+            float* pa = part_acc + item * D + sub * KV;
+#pragma unroll
+            for (int e = 0; e < KV; e += 4)
+                *reinterpret_cast<float4*>(pa + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+            if (sub == 0) part_ml[item] = make_float2(m, l);
+        }
     }
+}
+
+// out[r] = merge of the nparts partials in slots [r*nparts, (r+1)*nparts)
+template <class E>
+__global__ void __launch_bounds__(128) k_combine_rows(const float2* __restrict__ part_ml,
+                                                      const float* __restrict__ part_acc,
+                                                      typename E::T* __restrict__ out, int nparts,
+                                                      int D) {
+    const int64_t r = blockIdx.x;
+    const int c = threadIdx.x;
+    griddep_wait();  // partials come from the attention kernel
+    griddep_launch_dependents();
+    const float2* ml = part_ml + r * nparts;
+    float M = -INFINITY;
+    for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[p].x);
+    float L = 0.f, A = 0.f;
+    if (M != -INFINITY) {
+        for (int p = 0; p < nparts; ++p) {
+            const float sc = exp2f(ml[p].x - M);
+            L += ml[p].y * sc;
+            if (c < D) A += part_acc[(r * nparts + p) * D + c] * sc;
+        }
+    }
+    if (c < D) out[r * D + c] = E::from_float(L > 0.f ? A / L : 0.f);
 }
 
 template <class E>
@@ -166,23 +187,28 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)B * H_q;
-    const int64_t total = rows * k;
     auto kern = k_sparse_attn<E>;
-    const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0);
-    int64_t grid = (total + kSparseMinItems - 1) / kSparseMinItems;
-    if (grid > resident) grid = resident;
-    const int64_t per = (total + grid - 1) / grid;
-    grid = (total + per - 1) / per;
-    const int maxp = (int)((k - 1) / per + 2);
-    if (maxp > sparse_max_parts(k)) return cudaErrorInvalidValue;
+    const int64_t warps = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0) * 8;
+    int64_t nchunk = warps / rows;
+    if (nchunk < 1) nchunk = 1;
+    const int64_t cap = sparse_max_parts(rows, k);
+    if (nchunk > cap) nchunk = cap;
+    int64_t chunk = (k + nchunk - 1) / nchunk;
+    chunk = (chunk + kMinChunk - 1) / kMinChunk * kMinChunk;
+    nchunk = (k + chunk - 1) / chunk;
+    const int64_t n_items = rows * nchunk;
+    int64_t grid = (n_items + 7) / 8;
+    const int64_t max_grid = warps / 8;
+    if (grid > max_grid) grid = max_grid;
     using T = typename E::T;
     e = launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
                       static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv, (int)S,
-                      S_max, (int)k, scale * kLog2e, total, per, maxp, part_ml, part_acc);
+                      S_max, (int)k, scale * kLog2e, (int)chunk, (int)nchunk, n_items, part_ml,
+                      part_acc);
     if (e != cudaSuccess) return e;
-    return launch_kernel(k_combine<E>, dim3((unsigned)rows), dim3(128), 0, s, true,
-                         (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out), H_q,
-                         1, (int64_t)k, per, maxp, D);
+    return launch_kernel(k_combine_rows<E>, dim3((unsigned)rows), dim3(128), 0, s, true,
+                         (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out),
+                         (int)nchunk, D);
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,

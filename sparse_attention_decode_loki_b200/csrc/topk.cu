@@ -11,10 +11,12 @@
 // exact and deterministic.
 //
 // Rows of up to 32768 keys (k_topk_reg): each thread holds a contiguous run of
-// keys in registers. The first pass histograms the top 12 key bits (4096
-// shared-memory bins, sign + exponent + 3 mantissa bits), which already
-// isolates the threshold to a narrow bin; the next passes (10 + 10 bits) only
-// touch keys inside the chosen bin, so they cost a register scan each.
+// keys in registers. One block pass histograms the top 12 key bits (4096
+// shared-memory bins: sign, exponent and 3 mantissa bits), which already
+// narrows the threshold to one bin holding a few percent of the row; those
+// keys are gathered and warp 0 resolves the remaining 20 bits alone, with
+// ballot counts, so no further block barriers are paid. (A bin too crowded
+// for the gather buffer -- heavy ties -- takes two 10-bit block passes.)
 // Longer rows (k_topk_long) keep keys in shared memory, or re-read them from
 // L2 when they do not fit, with 8-bit digits and warp-aggregated atomics.
 #include "common.cuh"
@@ -58,42 +60,95 @@ __device__ __forceinline__ int block_excl_scan(int v, int* buf, int* total) {
 }
 
 // Given per-bin counts in hist[0, nbins) (bins ordered by key), find the bin
-// holding the krem-th largest counted key. Thread t owns bins [t*per, (t+1)*per).
-// Writes the bin to *s_bin and the rank left inside it to *s_krem.
+// holding the krem-th largest counted key. Thread t owns bins [t*per, (t+1)*per)
+// and reads them in a rotated order (bank-conflict free for per <= 32).
+// Writes the bin, the rank left inside it and the bin's count to shared memory.
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int krem, int* buf,
-                                         int* s_bin, int* s_krem) {
+                                         int* s_bin, int* s_krem, int* s_cnt) {
     const int per = nbins / (int)blockDim.x;
     const int b0 = threadIdx.x * per;
+    const int rot = threadIdx.x & (per - 1);
     int local = 0;
-    for (int i = 0; i < per; ++i) local += (int)hist[b0 + i];
+    for (int i = 0; i < per; ++i) local += (int)hist[b0 + ((i + rot) & (per - 1))];
     int total;
     const int before = block_excl_scan(local, buf, &total);
     int above = total - before - local;  // keys in bins owned by higher threads
-    for (int i = per - 1; i >= 0; --i) {
-        const int c = (int)hist[b0 + i];
-        if (above < krem && above + c >= krem) {
-            *s_bin = b0 + i;
-            *s_krem = krem - above;
+    if (above < krem && above + local >= krem) {
+        for (int i = per - 1; i >= 0; --i) {
+            const int c = (int)hist[b0 + i];
+            if (above < krem && above + c >= krem) {
+                *s_bin = b0 + i;
+                *s_krem = krem - above;
+                *s_cnt = c;
+            }
+            above += c;
         }
-        above += c;
     }
     __syncthreads();
+}
+
+// Warp-synchronous radix select over n candidate keys (all sharing their top
+// 12 bits) held in shared memory: finds the krem-th largest, 4 bits at a time
+// with ballots. Returns (low 20 bits of the threshold, rank left, its count).
+__device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int krem,
+                                              uint32_t* low, int* krem_out, int* cnt_out) {
+    const int lane = threadIdx.x & 31;
+    uint32_t prefix = 0u, mask = 0u;
+    int cnt_sel = 0;
+    for (int shift = 16; shift >= 0; shift -= 4) {
+        int cnt = 0;  // lane v < 16 counts digit v
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            const uint32_t c = i < n ? cand[i] : 0u;
+            const bool match = i < n && ((c & mask) == prefix);
+            const uint32_t dig = (c >> shift) & 15u;
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+                const unsigned m = __ballot_sync(0xffffffffu, match && dig == (uint32_t)v);
+                if (lane == v) cnt += __popc(m);
+            }
+        }
+        // suffix sums over digits (lanes 15 .. 0)
+        int suf = lane < 16 ? cnt : 0;
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1) {
+            const int y = __shfl_down_sync(0xffffffffu, suf, off);
+            if (lane + off < 16) suf += y;
+        }
+        const int above = suf - (lane < 16 ? cnt : 0);
+        const bool hit = lane < 16 && above < krem && above + cnt >= krem;
+        const unsigned hm = __ballot_sync(0xffffffffu, hit);
+        const int src = __ffs(hm) - 1;
+        const int a = __shfl_sync(0xffffffffu, above, src);
+        cnt_sel = __shfl_sync(0xffffffffu, cnt, src);
+        prefix |= (uint32_t)src << shift;
+        mask |= 15u << shift;
+        krem -= a;
+    }
+    *low = prefix;
+    *krem_out = krem;
+    *cnt_out = cnt_sel;
 }
 
 template <int KPT, int NT>
 __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ scores, int S, int k,
                                                  int32_t* __restrict__ out) {
+    constexpr int kCandCap = 2048;
     __shared__ uint32_t hist[4096];
+    __shared__ uint32_t cand[kCandCap];
     __shared__ int scan_buf[32];
-    __shared__ int s_bin, s_krem;
+    __shared__ int s_bin, s_krem, s_cnt, s_ncand;
+    __shared__ uint32_t s_T;
     const int tid = threadIdx.x;
     const float* row = scores + (int64_t)blockIdx.x * S;
     const int j0 = tid * KPT;
+    for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
+    if (tid == 0) s_ncand = 0;
     griddep_wait();  // scores come from the score kernel
     griddep_launch_dependents();
 
     uint32_t key[KPT];
-    if ((S & 3) == 0 && (KPT & 3) == 0) {
+    if ((S & 3) == 0) {
 #pragma unroll
         for (int e = 0; e < KPT; e += 4) {
             if (j0 + e < S) {
@@ -112,41 +167,66 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
     }
     // key 0 never comes from a score (NaN maps to the -inf key), so it marks
     // padding: it is never counted, selected or histogrammed
-
-    // pass 1: top 12 bits
-    for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
     __syncthreads();
+
+    // pass 1: top 12 bits over the whole row
 #pragma unroll
     for (int e = 0; e < KPT; ++e)
         if (key[e]) atomicAdd(&hist[key[e] >> 20], 1u);
     __syncthreads();
-    find_bin(hist, 4096, k, scan_buf, &s_bin, &s_krem);
+    find_bin(hist, 4096, k, scan_buf, &s_bin, &s_krem, &s_cnt);
     const uint32_t bin1 = (uint32_t)s_bin;
     int krem = s_krem;
-    __syncthreads();
+    const int n1 = s_cnt;  // keys in the threshold bin
 
-    // pass 2: bits 19..10 of the keys in bin1
-    for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
-    __syncthreads();
+    uint32_t T;
+    int cnt_T;
+    if (n1 <= kCandCap) {
+        // gather the threshold bin's keys; warp 0 resolves the low 20 bits
 #pragma unroll
-    for (int e = 0; e < KPT; ++e)
-        if (key[e] && (key[e] >> 20) == bin1) atomicAdd(&hist[(key[e] >> 10) & 1023u], 1u);
-    __syncthreads();
-    find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem);
-    const uint32_t pre2 = (bin1 << 10) | (uint32_t)s_bin;
-    krem = s_krem;
-    __syncthreads();
-
-    // pass 3: bits 9..0 of the keys matching the 22-bit prefix
-    for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
-    __syncthreads();
+        for (int e = 0; e < KPT; ++e)
+            if (key[e] && (key[e] >> 20) == bin1) cand[atomicAdd(&s_ncand, 1)] = key[e];
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t low;
+            int kr, c;
+            warp_select20(cand, s_ncand, krem, &low, &kr, &c);
+            if (tid == 0) {
+                s_T = (bin1 << 20) | low;
+                s_krem = kr;
+                s_cnt = c;
+            }
+        }
+        __syncthreads();
+        T = s_T;
+        krem = s_krem;
+        cnt_T = s_cnt;
+    } else {
+        // a crowded bin (heavy ties): two more block passes of 10 bits each
+        __syncthreads();
+        for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
+        __syncthreads();
 #pragma unroll
-    for (int e = 0; e < KPT; ++e)
-        if (key[e] && (key[e] >> 10) == pre2) atomicAdd(&hist[key[e] & 1023u], 1u);
-    __syncthreads();
-    find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem);
-    const uint32_t T = (pre2 << 10) | (uint32_t)s_bin;  // the k-th largest key
-    krem = s_krem;                                       // keys equal to T to take
+        for (int e = 0; e < KPT; ++e)
+            if (key[e] && (key[e] >> 20) == bin1) atomicAdd(&hist[(key[e] >> 10) & 1023u], 1u);
+        __syncthreads();
+        find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem, &s_cnt);
+        const uint32_t pre2 = (bin1 << 10) | (uint32_t)s_bin;
+        krem = s_krem;
+        __syncthreads();
+        for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < KPT; ++e)
+            if (key[e] && (key[e] >> 10) == pre2) atomicAdd(&hist[key[e] & 1023u], 1u);
+        __syncthreads();
+        find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem, &s_cnt);
+        T = (pre2 << 10) | (uint32_t)s_bin;
+        krem = s_krem;
+        cnt_T = s_cnt;
+    }
+    // T is the k-th largest key; krem of the cnt_T keys equal to T are taken,
+    // lowest indices first
 
     int gt = 0, eq = 0;
 #pragma unroll
@@ -154,9 +234,13 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
         gt += key[e] > T;
         eq += key[e] == T;
     }
-    int total;
-    const int eq_before = block_excl_scan(eq, scan_buf, &total);
-    const int take_eq = max(0, min(eq, krem - eq_before));
+    int total, take_eq;
+    if (krem == cnt_T) {
+        take_eq = eq;  // every key equal to T is selected: no tie scan needed
+    } else {
+        const int eq_before = block_excl_scan(eq, scan_buf, &total);
+        take_eq = max(0, min(eq, krem - eq_before));
+    }
     int pos = block_excl_scan(gt + take_eq, scan_buf, &total);
     int32_t* o = out + (int64_t)blockIdx.x * k;
     int eq_seen = 0;
@@ -265,10 +349,12 @@ static cudaError_t launch_reg(const float* scores, int64_t rows, int S, int k, i
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl) {
     const int Si = (int)S, ki = (int)k;
-    if (S <= 256 * 4) return launch_reg<4, 256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 8) return launch_reg<8, 256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 16) return launch_reg<16, 256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 512 * 16) return launch_reg<16, 512>(scores, rows, Si, ki, idx, s, pdl);
+    // find_bin needs 4096 and 1024 bins to split evenly over the threads (NT <= 1024)
+    if (S <= 128 * 4) return launch_reg<4, 128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 128 * 8) return launch_reg<8, 128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 128 * 16) return launch_reg<16, 128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 128 * 32) return launch_reg<32, 128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 32) return launch_reg<32, 256>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 512 * 32) return launch_reg<32, 512>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 512 * 64) return launch_reg<64, 512>(scores, rows, Si, ki, idx, s, pdl);
     {
