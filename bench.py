@@ -293,7 +293,7 @@ def run_ours(args):
         @staticmethod
         def zero_():
             flush_w.zero_()
-            torch.sum(flush_r, out=flush_sink)
+            torch.sum(flush_r, dim=0, out=flush_sink)
 
     flush = _Flush()
 
