@@ -13,7 +13,7 @@ LIB_PATH = os.path.join(_HERE, "libloki.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m sparse_attention_decode_loki_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python sparse_attention_decode_loki_b200/build.py`"
     )
 
 lib = ctypes.CDLL(LIB_PATH)

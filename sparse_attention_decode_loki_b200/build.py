@@ -1,6 +1,9 @@
 """Build libloki.so in-tree with nvcc for sm_100a.
 
-    python -m sparse_attention_decode_loki_b200.build [--verbose]
+    python sparse_attention_decode_loki_b200/build.py [--verbose] [--force]
+
+(Run it as a file, not as `-m`: importing the package loads libloki.so, which
+is what this script produces.)
 
 Each .cu under csrc/ compiles to an object in _build/ (in parallel), then the
 objects link into sparse_attention_decode_loki_b200/libloki.so with the CUDA
