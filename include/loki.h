@@ -160,6 +160,26 @@ LOKI_API loki_status loki_decode_attention_plane(const void* q, const void* Kt_c
                                                  int32_t* selected_idx, void* ws, size_t ws_bytes,
                                                  void* stream);
 
+/*
+ * loki_decode_attention without a workspace argument, for callers that cannot
+ * allocate device memory (a plugin inside a framework that owns all device
+ * allocations, a thread that must not call cudaMalloc/cudaFree because they
+ * can synchronise the device). The paper has no counterpart: this is a
+ * memory-management convenience of this library. Scratch comes from a
+ * 32 MiB array built into the library (held on every GPU that loads it until
+ * the process exits); a decode that needs more (loki_decode_workspace_size)
+ * returns LOKI_ERR_UNSUPPORTED without launching anything. All calls share
+ * the array, so calls that overlap on the GPU race. The first call on each
+ * device looks up the array's address; make it before any stream capture.
+ * Other arguments and results are those of loki_decode_attention.
+ */
+LOKI_API loki_status loki_decode_attention_noalloc(const void* q, const void* Kt_cache,
+                                                   const void* V_cache, const float* P, int B,
+                                                   int H_q, int H_kv, int64_t S, int64_t S_max,
+                                                   int D, int d, int64_t k, float scale,
+                                                   loki_dtype dt, void* out, int32_t* selected_idx,
+                                                   void* stream);
+
 /* Steps of loki_decode_attention, callable one by one ------------------- */
 
 /* q_rot [B, H_q, D] fp32 = q P (query rotated into its KV head's basis). */

@@ -41,6 +41,9 @@ PROTOTYPES = {
                                             c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,
                                             c_int, c_int64, c_float, c_int, c_void_p, c_void_p,
                                             c_void_p, c_size_t, c_void_p]),
+    "loki_decode_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                              c_int, c_int64, c_int64, c_int, c_int, c_int64,
+                                              c_float, c_int, c_void_p, c_void_p, c_void_p]),
     "loki_project_query": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p,
                                    c_void_p]),
     "loki_score_lowdim": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,

@@ -163,6 +163,10 @@ T* at(void* base, size_t off) {
 
 }  // namespace
 
+namespace loki {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace loki
+
 extern "C" {
 
 const char* loki_status_string(loki_status st) {

@@ -21,6 +21,9 @@ cudaError_t dev_info(DevInfo* out);
 // resident CTAs per SM of `func` at `threads` threads and `smem` dynamic bytes (cached)
 int occupancy(const void* func, int threads, size_t smem);
 
+// sets the text loki_last_error() returns on the calling thread
+void set_last_error(const char* msg);
+
 // ---- decode steps --------------------------------------------------------
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
                                  int D, float* q_rot, cudaStream_t s);
