@@ -69,6 +69,14 @@ LOKI_API const char* loki_status_string(loki_status st);
 /* Description of the last failure on the calling thread ("" if none). */
 LOKI_API const char* loki_last_error(void);
 
+/*
+ * Kernel error word of the current device: nonzero (1) if a staged kernel's
+ * bounded wait on an asynchronous copy gave up (its results are then
+ * invalid). Synchronous: copies 4 bytes from the device (waiting for prior
+ * work); with reset != 0 the word is cleared afterwards.
+ */
+LOKI_API loki_status loki_device_error(int* code, int reset);
+
 /* ------------------------------------------------------------------------ */
 /* Offline calibration                                                      */
 /* ------------------------------------------------------------------------ */

@@ -26,8 +26,16 @@ __all__ = [
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
     "loki_sparse_attention_workspace_size", "loki_calibrate_workspace_size",
-    "loki_topk_workspace_size",
+    "loki_topk_workspace_size", "loki_device_error",
 ]
+
+
+def loki_device_error(reset: bool = False) -> int:
+    """Kernel error word of the current device (0 = no staged wait gave up)."""
+    import ctypes
+    code = ctypes.c_int(0)
+    check(lib.loki_device_error(ctypes.byref(code), int(reset)), "loki_device_error")
+    return code.value
 
 
 def _dt(t: torch.Tensor) -> int:

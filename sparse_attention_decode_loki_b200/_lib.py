@@ -25,6 +25,7 @@ c_void_p, c_char_p = ctypes.c_void_p, ctypes.c_char_p
 PROTOTYPES = {
     "loki_status_string": (c_char_p, [c_int]),
     "loki_last_error": (c_char_p, []),
+    "loki_device_error": (c_int, [ctypes.POINTER(c_int), c_int]),
     "loki_calibrate_workspace_size": (c_size_t, [c_int64, c_int, c_int]),
     "loki_calibrate_pca": (c_int, [c_void_p, c_int, c_int64, c_int, c_int, c_void_p, c_void_p,
                                    c_void_p, c_size_t, c_void_p]),

@@ -104,7 +104,7 @@ float resolve_scale(float scale, int D) {
 
 // workspace pieces of the decode path
 struct DecodeWs {
-    size_t q_rot, scores, ml, acc, total;
+    size_t q_rot, scores, done, ml, acc, total;
 };
 DecodeWs decode_ws(int B, int H_q, int64_t S, int D, int64_t k) {
     const int64_t rows = (int64_t)B * H_q;
@@ -112,21 +112,23 @@ DecodeWs decode_ws(int B, int H_q, int64_t S, int D, int64_t k) {
     DecodeWs w;
     w.q_rot = 0;
     w.scores = align_up(w.q_rot + (size_t)rows * D * sizeof(float));
-    w.ml = align_up(w.scores + (size_t)rows * S * sizeof(float));
+    w.done = align_up(w.scores + (size_t)rows * S * sizeof(float));
+    w.ml = align_up(w.done + (size_t)rows * sizeof(int));
     w.acc = align_up(w.ml + (size_t)rows * parts * sizeof(float2));
     w.total = align_up(w.acc + (size_t)rows * parts * D * sizeof(float));
     return w;
 }
 
 struct SparseWs {
-    size_t ml, acc, total;
+    size_t done, ml, acc, total;
 };
 SparseWs sparse_ws(int B, int H_q, int64_t k, int D) {
     const int64_t rows = (int64_t)B * H_q;
     const int64_t parts = loki::sparse_max_parts(rows, k);
     SparseWs w;
-    w.ml = 0;
-    w.acc = align_up((size_t)rows * parts * sizeof(float2));
+    w.done = 0;
+    w.ml = align_up((size_t)rows * sizeof(int));
+    w.acc = align_up(w.ml + (size_t)rows * parts * sizeof(float2));
     w.total = align_up(w.acc + (size_t)rows * parts * D * sizeof(float));
     return w;
 }
@@ -181,6 +183,16 @@ const char* loki_status_string(loki_status st) {
 }
 
 const char* loki_last_error(void) { return g_last_error.c_str(); }
+
+loki_status loki_device_error(int* code, int reset) {
+    g_last_error.clear();
+    LOKI_REQUIRE(code != nullptr, LOKI_ERR_INVALID_ARG, "code must not be NULL");
+    int* w = loki::device_error_word();
+    LOKI_REQUIRE(w != nullptr, LOKI_ERR_CUDA, "no usable current CUDA device");
+    LOKI_CUDA(cudaMemcpy(code, w, sizeof(int), cudaMemcpyDeviceToHost), "loki_device_error");
+    if (reset) LOKI_CUDA(cudaMemset(w, 0, sizeof(int)), "loki_device_error");
+    return LOKI_OK;
+}
 
 // ---------------------------------------------------------------------------
 
@@ -304,21 +316,28 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
     const loki::Dt t = to_dt(dt);
     float* q_rot = at<float>(ws, w.q_rot);
     float* scores = at<float>(ws, w.scores);
-    // The first kernel is ordered normally after whatever precedes the call;
-    // the later ones use programmatic dependent launch.
-    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), name);
+    int* done = at<int>(ws, w.done);
+    const int rows = B * H_q;
+    // Four kernels: query projection (which also zeroes the attention
+    // kernel's row counters); score scan (over a low-dim key plane the
+    // TMA-staged scan, which starts streaming keys while the projection runs;
+    // over the row layout the register-staged scan); top-k; attention with
+    // its row merge. The first kernel is ordered normally after whatever
+    // precedes the call; the later ones use programmatic dependent launch.
+    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows), name);
     if (Kt_lo != nullptr)
-        LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
-                                            scores, s, true),
+        LOKI_CUDA(loki::launch_score_plane(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
+                                           scores, s, true),
                   name);
     else
         LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, D, d,
                                             scores, s, true),
                   name);
-    LOKI_CUDA(loki::launch_topk(scores, (int64_t)B * H_q, S, k, selected_idx, s, true), name);
+    LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
-                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), s, true),
+                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
+                                            true),
               name);
     return LOKI_OK;
 }
@@ -428,10 +447,13 @@ loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, cons
     const SparseWs w = sparse_ws(B, H_q, k, D);
     LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
                  "workspace %zu bytes < required %zu", ws_bytes, w.total);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LOKI_CUDA(cudaMemsetAsync(at<int>(ws, w.done), 0, (size_t)B * H_q * sizeof(int), s),
+              "sparse_attention");
     LOKI_CUDA(loki::launch_sparse_attention(to_dt(dt), q_rot, Kt_cache, V_cache, selected_idx, B,
                                             H_q, H_kv, S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc),
-                                            static_cast<cudaStream_t>(stream), false),
+                                            at<int>(ws, w.done), s, false),
               "sparse_attention");
     return LOKI_OK;
 }

@@ -21,12 +21,17 @@ cudaError_t dev_info(DevInfo* out);
 // resident CTAs per SM of `func` at `threads` threads and `smem` dynamic bytes (cached)
 int occupancy(const void* func, int threads, size_t smem);
 
+// device address of this device's kernel error word (cached; null on failure)
+int* device_error_word();
+
 // sets the text loki_last_error() returns on the calling thread
 void set_last_error(const char* msg);
 
 // ---- decode steps --------------------------------------------------------
+// also zeroes done[0, n_done) when done is not null
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
-                                 int D, float* q_rot, cudaStream_t s);
+                                 int D, float* q_rot, cudaStream_t s, int* done = nullptr,
+                                 int n_done = 0);
 
 // `row` is the row length (and stride) of the key buffer scanned: D for the
 // rotated cache, d_lo for a low-dimensional key plane.
@@ -34,15 +39,25 @@ cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B
                                 int H_kv, int64_t S, int64_t S_max, int D, int row, int d,
                                 float* scores, cudaStream_t s, bool pdl);
 
+// TMA-staged scan of a low-dim key plane Klo [B, H_kv, S_max, d_lo]. With pdl
+// it may start while the projection that writes q_rot is still running (it
+// streams keys first, then waits).
+cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
+                               int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
+                               float* scores, cudaStream_t s, bool pdl);
+
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl);
 
 // partial slots per (batch, query head) row of the sparse attention split
 int64_t sparse_max_parts(int64_t rows, int64_t k);
+// done[B*H_q] must be zero on entry (per-row completion counters; the last
+// warp of a row merges its partials into out and leaves the counter at zero).
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
-                                    float2* part_ml, float* part_acc, cudaStream_t s, bool pdl);
+                                    float2* part_ml, float* part_acc, int* done, cudaStream_t s,
+                                    bool pdl);
 
 // split-S partial slots per (batch, KV head) unit
 int64_t dense_max_parts(int64_t S);

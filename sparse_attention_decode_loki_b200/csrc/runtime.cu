@@ -9,8 +9,13 @@
 
 namespace loki {
 
+// Set by a kernel whose bounded wait on an asynchronous copy gave up (see
+// tma.cuh); read and cleared through loki_device_error().
+__device__ int g_device_error;
+
 namespace {
 constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {};
 std::mutex g_mu;
 DevInfo g_dev[kMaxDevices];
 bool g_dev_ok[kMaxDevices] = {};
@@ -49,6 +54,18 @@ cudaError_t dev_info(DevInfo* out) {
     }
     *out = g_dev[dev];
     return cudaSuccess;
+}
+
+int* device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_err_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_err_ptr[dev];
 }
 
 int occupancy(const void* func, int threads, size_t smem) {

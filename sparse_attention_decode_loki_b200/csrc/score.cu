@@ -1,4 +1,4 @@
-// Query rotation and the low-dimensional score scan of Loki.
+// Query rotation and the (register-staged) low-dimensional score scan of Loki.
 //
 // Loki (NeurIPS 2024 poster page, TL;DR and "Visual Insights" Figure 1
 // caption; briefgpt.xyz abstract page): the query is projected onto the PCA
@@ -16,7 +16,8 @@
 
 namespace loki {
 
-// q_rot[row, c] = sum_i q[row, i] P[h_kv, i, c]. One CTA per (KV head, block of
+// q_rot[row, c] = sum_i q[row, i] P[h_kv, i, c]; also zeroes done[0, n_done)
+// (the attention kernel's per-row counters) when done is given. One CTA per (KV head, block of
 // 32 output columns, chunk of up to 32 query rows of that head): the P column
 // block (128 x 32 fp32) is staged once in shared memory and reused by every
 // query of the head; each warp computes one query's 32 columns per step.
@@ -27,9 +28,17 @@ template <class E>
 __global__ void __launch_bounds__(256) k_project_query(const typename E::T* __restrict__ q,
                                                        const float* __restrict__ P,
                                                        float* __restrict__ q_rot, int B, int H_q,
-                                                       int G, int D) {
+                                                       int G, int D, int* __restrict__ done,
+                                                       int n_done) {
     __shared__ float Ps[128][kProjCols];
     __shared__ float qs[kProjRows][128];
+    // the next kernel (the score scan) may start streaming keys right away
+    griddep_launch_dependents();
+    if (done != nullptr) {
+        const int nb = gridDim.x * gridDim.y * gridDim.z;
+        const int bid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+        for (int i = bid * 256 + (int)threadIdx.x; i < n_done; i += nb * 256) done[i] = 0;
+    }
     const int hk = blockIdx.x;
     const int c0 = blockIdx.y * kProjCols;
     const int r0 = blockIdx.z * kProjRows;
@@ -114,11 +123,12 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
         const int seg = (int)min64(r_end - r, (int64_t)S - s0);
         const int b = (int)(unit / H_kv);
         const int hk = (int)(unit % H_kv);
+        const int64_t qrow0 = (int64_t)b * H_q + (int64_t)hk * G;
 
         float qv[G][KV];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float* qp = q_rot + ((int64_t)b * H_q + (int64_t)hk * G + g) * D + sub * KV;
+            const float* qp = q_rot + (qrow0 + g) * D + sub * KV;
 #pragma unroll
             for (int e = 0; e < KV; ++e) {
                 const int col = sub * KV + e;
@@ -127,7 +137,7 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
         }
         const char* base =
             reinterpret_cast<const char*>(Kt) + (unit * S_max + s0) * row_bytes + sub * 16;
-        float* srow = scores + ((int64_t)b * H_q + (int64_t)hk * G) * S + s0;
+        float* srow = scores + qrow0 * S + s0;
 
         for (int p = 0; p < seg; p += rows_per_pass * U) {
             uint4 v[U];
@@ -159,15 +169,15 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
 }
 
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
-                                 int D, float* q_rot, cudaStream_t s) {
+                                 int D, float* q_rot, cudaStream_t s, int* done, int n_done) {
     const int G = H_q / H_kv;
     dim3 grid(H_kv, (D + kProjCols - 1) / kProjCols, (B * G + kProjRows - 1) / kProjRows);
     if (dt == kF32)
         k_project_query<ElemF32><<<grid, 256, 0, s>>>(static_cast<const float*>(q), P, q_rot, B,
-                                                      H_q, G, D);
+                                                      H_q, G, D, done, n_done);
     else
         k_project_query<ElemBF16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), P,
-                                                       q_rot, B, H_q, G, D);
+                                                       q_rot, B, H_q, G, D, done, n_done);
     return cudaGetLastError();
 }
 

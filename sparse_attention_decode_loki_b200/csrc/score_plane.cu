@@ -1,0 +1,250 @@
+// Low-dimensional score scan over a low-dim key plane, staged through shared
+// memory by TMA bulk copies.
+//
+// Loki (NeurIPS 2024 poster page, TL;DR and "Visual Insights" Figure 1
+// caption; briefgpt.xyz abstract page): every cached token is scored on the
+// first d principal components, s_j = q~[:d] . K~_j[:d], with q~ = q P.
+//
+// A (batch, KV head) unit's plane rows are contiguous (d_lo elements each),
+// so the scan is a pure stream. The rows of all units are laid end to end and
+// split evenly over one wave of CTAs. In each CTA one producer warp issues
+// cp.async.bulk copies of 256-row tiles into a 96 KB ring of shared-memory
+// stages (full/empty mbarriers); each of 256 consumer threads scores one row
+// of every tile for all G query heads of the unit (whole row per thread: no
+// shuffles, coalesced score stores), reading the row's 16-byte chunks in a
+// rotated order so a quarter-warp touches distinct banks. The ring keeps up
+// to ~90 KB per SM in flight without holding it in registers. Launched right behind the query
+// projection (programmatic dependent launch): the producer starts streaming
+// keys at once, and only the consumers wait for the projection's q~.
+#include "common.cuh"
+#include "launch.h"
+#include "tma.cuh"
+
+namespace loki {
+
+constexpr int kScoreConsumerWarps = 8;
+constexpr int kScoreConsumers = kScoreConsumerWarps * 32;
+constexpr int kScoreThreads = kScoreConsumers + 32;
+// one CTA per SM (9 warps at ~104 registers leave no room for a second);
+// a 192 KB ring measured no faster than this one
+constexpr int kScoreRingBytes = 96 * 1024;
+constexpr int kScoreMaxStages = 16;
+
+// NV = 16-byte chunks per plane row (d_lo * elem / 16). A tile is 256 rows,
+// one per consumer thread; stages = ring bytes / tile bytes.
+template <class E, int G, int NV>
+__global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
+    const float* __restrict__ q_rot, const typename E::T* __restrict__ Klo,
+    float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
+    int D, int d, int64_t total, int64_t per) {
+    constexpr int KV = E::kVec;
+    constexpr int kRowBytes = NV * 16;
+    constexpr int kTR = kScoreConsumers;  // rows per tile
+    constexpr int kTile = kTR * kRowBytes;
+    constexpr int kStages = (kScoreRingBytes / kTile) < kScoreMaxStages ? (kScoreRingBytes / kTile)
+                                                                      : kScoreMaxStages;
+    static_assert(kStages >= 2, "ring too small");
+    extern __shared__ __align__(128) unsigned char ring[];
+    __shared__ uint64_t full[kStages], empty[kStages];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kScoreConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    griddep_launch_dependents();
+
+    const int64_t R0 = (int64_t)blockIdx.x * per;
+    const int64_t R1 = min64(R0 + per, total);
+
+    if (warp == kScoreConsumerWarps) {
+        // ---------------- producer: one lane issues every tile copy ----------------
+        if (lane == 0) {
+            int i = 0;
+            bool ok = true;
+            for (int64_t r = R0; r < R1 && ok;) {
+                const int64_t unit = r / S;
+                const int s0 = (int)(r - unit * S);
+                const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+                const char* src = reinterpret_cast<const char*>(Klo) + (unit * S_max + s0) * kRowBytes;
+                for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
+                    const int n = min(kTR, seg - t0);
+                    const int st = i % kStages;
+                    const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+                    if (!mbar_wait(&empty[st], ph ^ 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[st], (uint32_t)(n * kRowBytes));
+                    bulk_load(ring + (size_t)st * kTile, src + (int64_t)t0 * kRowBytes,
+                              (uint32_t)(n * kRowBytes), &full[st]);
+                }
+                r += seg;
+            }
+            // every issued copy has landed before the CTA may exit
+            for (int j = max(0, i - kStages); j < i; ++j)
+                mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, err);
+        }
+        return;
+    }
+
+    // ---------------- consumers: one row of each tile per thread ----------------
+    // q~ comes from the projection kernel, which may still be running: the
+    // producer above streams keys without waiting, the consumers wait here.
+    griddep_wait();
+    // chunk c of a row is read at rotation (c + tid / 2) % NV: the 8 threads
+    // of a quarter-warp then hit 8 distinct 16-byte bank groups
+    const int rot = (tid >> 1) & (NV - 1);
+    bool bad = false;
+    int i = 0;
+    for (int64_t r = R0; r < R1;) {
+        const int64_t unit = r / S;
+        const int s0 = (int)(r - unit * S);
+        const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+        const int b = (int)(unit / H_kv), hk = (int)(unit % H_kv);
+        const int64_t qrow0 = (int64_t)b * H_q + (int64_t)hk * G;
+        // qv holds q~ in this thread's rotated chunk order: slot cc holds
+        // chunk (cc + rot) % NV, so the row loop indexes registers statically
+        float qv[G][NV * KV];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int cc = 0; cc < NV; ++cc)
+#pragma unroll
+                for (int e = 0; e < KV; ++e) {
+                    const int col = ((cc + rot) & (NV - 1)) * KV + e;
+                    qv[g][cc * KV + e] = col < d ? __ldg(q_rot + (qrow0 + g) * D + col) : 0.f;
+                }
+
+        float* srow = scores + qrow0 * S + s0;
+        for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
+            const int n = min(kTR, seg - t0);
+            const int st = i % kStages;
+            const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+            // after a timed-out wait this warp stops consuming and stops
+            // releasing stages, so the producer stops issuing and drains
+            if (!bad && !mbar_wait(&full[st], ph, err)) bad = true;
+            if (!bad && tid < n) {
+                const unsigned char* rowp = ring + (size_t)st * kTile + tid * kRowBytes;
+                float a[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) a[g] = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < NV; ++cc) {
+                    const int c = (cc + rot) & (NV - 1);
+                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + c * 16);
+                    float f[KV];
+                    E::unpack(v, f);
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int e = 0; e < KV; ++e) a[g] = fmaf(qv[g][cc * KV + e], f[e], a[g]);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) srow[(int64_t)g * S + t0 + tid] = a[g];
+            }
+            __syncwarp();
+            if (lane == 0 && !bad) mbar_arrive(&empty[st]);
+        }
+        r += seg;
+    }
+}
+
+template <class E, int G, int NV>
+static cudaError_t plane_impl(const float* q_rot, const void* Klo, float* scores, int* err, int B,
+                              int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                              cudaStream_t s, bool pdl) {
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    constexpr int kTile = kScoreConsumers * NV * 16;
+    constexpr int kStages = (kScoreRingBytes / kTile) < kScoreMaxStages ? (kScoreRingBytes / kTile)
+                                                                      : kScoreMaxStages;
+    auto kern = k_score_plane<E, G, NV>;
+    const size_t smem = (size_t)kStages * kTile;
+    static bool attr_set[64] = {};
+    if (di.device < 64 && !attr_set[di.device]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[di.device] = true;
+    }
+    const int64_t total = (int64_t)B * H_kv * S;
+    const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, kScoreThreads, smem);
+    int64_t grid = (total + kScoreConsumers - 1) / kScoreConsumers;
+    if (grid > resident) grid = resident;
+    const int64_t per = (total + grid - 1) / grid;
+    grid = (total + per - 1) / per;
+    using T = typename E::T;
+    return launch_kernel(kern, dim3((unsigned)grid), dim3(kScoreThreads), smem, s, pdl, q_rot,
+                         static_cast<const T*>(Klo), scores, err, H_q, H_kv, (int)S, S_max, D, d,
+                         total, per);
+}
+
+template <class E, int G, int NV>
+static cudaError_t plane_if(const float* q_rot, const void* Klo, float* scores, int* err, int B,
+                            int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                            cudaStream_t s, bool pdl) {
+    if constexpr (G * NV * E::kVec <= 64)
+        return plane_impl<E, G, NV>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+    else
+        return cudaErrorInvalidValue;  // not dispatched (see score_plane_supported)
+}
+
+template <class E, int G>
+static cudaError_t plane_nv(int nv, const float* q_rot, const void* Klo, float* scores, int* err,
+                            int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                            cudaStream_t s, bool pdl) {
+    switch (nv) {
+        case 1: return plane_if<E, G, 1>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        case 2: return plane_if<E, G, 2>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        case 4: return plane_if<E, G, 4>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        case 8: return plane_if<E, G, 8>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <class E>
+static cudaError_t plane_dispatch(int G, int nv, const float* q_rot, const void* Klo,
+                                  float* scores, int* err, int B, int H_q, int H_kv, int64_t S,
+                                  int64_t S_max, int D, int d, cudaStream_t s, bool pdl) {
+    switch (G) {
+#define LOKI_G(g)                                                                              \
+    case g:                                                                                    \
+        return plane_nv<E, g>(nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
+#undef LOKI_G
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// Plane rows of 1, 2, 4 or 8 chunks with G * chunks * elements <= 64 take the
+// thread-per-row TMA kernel; other planes take the register-staged scan.
+bool score_plane_supported(Dt dt, int G, int d_lo) {
+    const int row_bytes = d_lo * (dt == kF32 ? 4 : 2);
+    const int nv = row_bytes / 16;
+    const int kv = dt == kF32 ? 4 : 8;
+    return row_bytes % 16 == 0 && (nv == 1 || nv == 2 || nv == 4 || nv == 8) && G * nv * kv <= 64;
+}
+
+cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
+                               int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
+                               float* scores, cudaStream_t s, bool pdl) {
+    int* err = device_error_word();
+    if (err == nullptr) return cudaErrorInvalidDevice;
+    const int G = H_q / H_kv;
+    if (!score_plane_supported(dt, G, d_lo))
+        return launch_score_lowdim(dt, q_rot, Klo, B, H_q, H_kv, S, S_max, D, d_lo, d, scores, s,
+                                   pdl);
+    const int nv = d_lo * (dt == kF32 ? 4 : 2) / 16;
+    if (dt == kF32)
+        return plane_dispatch<ElemF32>(G, nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D,
+                                       d, s, pdl);
+    return plane_dispatch<ElemBF16>(G, nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d,
+                                    s, pdl);
+}
+
+}  // namespace loki

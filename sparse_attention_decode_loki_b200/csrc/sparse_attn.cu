@@ -9,8 +9,9 @@
 // matching value row per step, 8 rows in flight; every row is a random but
 // contiguous gather. Scores use all D dimensions in fp32; the softmax runs
 // online in base 2 with the scale folded into q~. The warp merges its row
-// groups with shuffles and writes one partial; k_combine_rows merges a row's
-// partials.
+// groups with shuffles and writes one partial; the last warp to finish a row
+// (a per-row atomic counter) merges that row's partials into the output, so
+// no separate combine kernel runs.
 #include "common.cuh"
 #include "launch.h"
 
@@ -27,7 +28,7 @@ int64_t sparse_max_parts(int64_t rows, int64_t k) {
     int64_t cap = 10240 / rows;
     if (cap < 1) cap = 1;
     const int64_t by_k = (k + kMinChunk - 1) / kMinChunk;
-    return by_k < cap ? by_k : cap;
+    return (by_k < cap ? by_k : cap) + 2;
 }
 
 template <class E>
@@ -35,7 +36,8 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int chunk, int nchunk, int64_t n_items,
-    float2* __restrict__ part_ml, float* __restrict__ part_acc) {
+    float2* __restrict__ part_ml, float* __restrict__ part_acc, int* __restrict__ done,
+    typename E::T* __restrict__ out) {
     constexpr int D = 128;
     constexpr int KV = E::kVec;
     constexpr int LPR = D / KV;     // lanes per row
@@ -151,38 +153,46 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
                 *reinterpret_cast<float4*>(pa + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
             if (sub == 0) part_ml[item] = make_float2(m, l);
         }
-    }
-}
-
-// out[r] = merge of the nparts partials in slots [r*nparts, (r+1)*nparts)
-template <class E>
-__global__ void __launch_bounds__(128) k_combine_rows(const float2* __restrict__ part_ml,
-                                                      const float* __restrict__ part_acc,
-                                                      typename E::T* __restrict__ out, int nparts,
-                                                      int D) {
-    const int64_t r = blockIdx.x;
-    const int c = threadIdx.x;
-    griddep_wait();  // partials come from the attention kernel
-    griddep_launch_dependents();
-    const float2* ml = part_ml + r * nparts;
-    float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, ml[p].x);
-    float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-        for (int p = 0; p < nparts; ++p) {
-            const float sc = exp2f(ml[p].x - M);
-            L += ml[p].y * sc;
-            if (c < D) A += part_acc[(r * nparts + p) * D + c] * sc;
+        // The last warp to finish a chunk of row r merges the row's partials
+        // (its own included) into out[r]: publish, count, and only the warp
+        // that sees the count reach nchunk reads the others' partials.
+        __threadfence();  // each lane's partial writes are visible device-wide...
+        __syncwarp();     // ...before lane 0 counts the chunk as done
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(done + r, 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == nchunk - 1) {
+            __threadfence();
+            const float2* ml = part_ml + r * nchunk;
+            float M = -INFINITY;
+            for (int p = 0; p < nchunk; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
+            float Lsum = 0.f, A[D / 32];
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) A[e] = 0.f;
+            if (M != -INFINITY) {
+                for (int p = 0; p < nchunk; ++p) {
+                    const float2 mlp = __ldcg(&ml[p]);
+                    const float sc = exp2f(mlp.x - M);
+                    Lsum += mlp.y * sc;
+                    const float* pa = part_acc + (r * nchunk + p) * D;
+#pragma unroll
+                    for (int e = 0; e < D / 32; ++e) A[e] += __ldcg(pa + e * 32 + lane) * sc;
+                }
+            }
+            const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) out[r * D + e * 32 + lane] = E::from_float(A[e] * inv);
+            if (lane == 0) done[r] = 0;  // leave the counter ready for the next call
         }
     }
-    if (c < D) out[r * D + c] = E::from_float(L > 0.f ? A / L : 0.f);
 }
 
 template <class E>
 static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V,
                                const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                int64_t S_max, int D, int64_t k, float scale, void* out,
-                               float2* part_ml, float* part_acc, cudaStream_t s, bool pdl) {
+                               float2* part_ml, float* part_acc, int* done, cudaStream_t s,
+                               bool pdl) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
@@ -201,25 +211,22 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     const int64_t max_grid = warps / 8;
     if (grid > max_grid) grid = max_grid;
     using T = typename E::T;
-    e = launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
-                      static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv, (int)S,
-                      S_max, (int)k, scale * kLog2e, (int)chunk, (int)nchunk, n_items, part_ml,
-                      part_acc);
-    if (e != cudaSuccess) return e;
-    return launch_kernel(k_combine_rows<E>, dim3((unsigned)rows), dim3(128), 0, s, true,
-                         (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out),
-                         (int)nchunk, D);
+    return launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
+                         static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv,
+                         (int)S, S_max, (int)k, scale * kLog2e, (int)chunk, (int)nchunk, n_items,
+                         part_ml, part_acc, done, static_cast<T*>(out));
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
-                                    float2* part_ml, float* part_acc, cudaStream_t s, bool pdl) {
+                                    float2* part_ml, float* part_acc, int* done, cudaStream_t s,
+                                    bool pdl) {
     if (dt == kF32)
         return sparse_impl<ElemF32>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                    part_ml, part_acc, s, pdl);
+                                    part_ml, part_acc, done, s, pdl);
     return sparse_impl<ElemBF16>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                 part_ml, part_acc, s, pdl);
+                                 part_ml, part_acc, done, s, pdl);
 }
 
 }  // namespace loki

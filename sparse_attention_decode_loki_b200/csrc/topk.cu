@@ -14,8 +14,9 @@
 // keys in registers. One block pass histograms the top 12 key bits (4096
 // shared-memory bins: sign, exponent and 3 mantissa bits), which already
 // narrows the threshold to one bin holding a few percent of the row; those
-// keys are gathered and warp 0 resolves the remaining 20 bits alone, with
-// ballot counts, so no further block barriers are paid. (A bin too crowded
+// keys are gathered and warp 0 resolves the remaining 20 bits alone with two
+// 10-bit passes over a warp-private histogram, so no further block barriers
+// are paid. (A bin too crowded
 // for the gather buffer -- heavy ties -- takes two 10-bit block passes.)
 // Longer rows (k_topk_long) keep keys in shared memory, or re-read them from
 // L2 when they do not fit, with 8-bit digits and warp-aggregated atomics.
@@ -87,45 +88,57 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int kr
     __syncthreads();
 }
 
-// Warp-synchronous radix select over n candidate keys (all sharing their top
-// 12 bits) held in shared memory: finds the krem-th largest, 4 bits at a time
-// with ballots. Returns (low 20 bits of the threshold, rank left, its count).
-__device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int krem,
+// Warp-synchronous select over n candidate keys (all sharing their top 12
+// bits) held in shared memory: finds the krem-th largest with two 10-bit
+// passes over a warp-private 1024-bin histogram `h`. Lane l owns bins
+// [32l, 32l + 32) and reads them rotated by l (bank-conflict free). Returns
+// (low 20 bits of the threshold, rank left inside it, count of keys equal to it).
+__device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int krem, uint32_t* h,
                                               uint32_t* low, int* krem_out, int* cnt_out) {
     const int lane = threadIdx.x & 31;
-    uint32_t prefix = 0u, mask = 0u;
+    uint32_t hi10 = 0u;
     int cnt_sel = 0;
-    for (int shift = 16; shift >= 0; shift -= 4) {
-        int cnt = 0;  // lane v < 16 counts digit v
-        for (int base = 0; base < n; base += 32) {
-            const int i = base + lane;
-            const uint32_t c = i < n ? cand[i] : 0u;
-            const bool match = i < n && ((c & mask) == prefix);
-            const uint32_t dig = (c >> shift) & 15u;
 #pragma unroll
-            for (int v = 0; v < 16; ++v) {
-                const unsigned m = __ballot_sync(0xffffffffu, match && dig == (uint32_t)v);
-                if (lane == v) cnt += __popc(m);
+    for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[32 * i + lane] = 0u;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t c = cand[i];
+            if (pass == 0 || ((c >> 10) & 1023u) == hi10) atomicAdd(&h[(c >> shift) & 1023u], 1u);
+        }
+        __syncwarp();
+        int local = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) local += (int)h[32 * lane + ((i + lane) & 31)];
+        int suf = local;  // inclusive suffix sum over lanes
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_down_sync(0xffffffffu, suf, off);
+            if (lane + off < 32) suf += y;
+        }
+        int above = suf - local;
+        int bin = -1, kr = 0, cnt = 0;
+        if (above < krem && above + local >= krem) {
+            for (int i = 31; i >= 0; --i) {
+                const int c = (int)h[32 * lane + i];
+                if (above < krem && above + c >= krem) {
+                    bin = 32 * lane + i;
+                    kr = krem - above;
+                    cnt = c;
+                }
+                above += c;
             }
         }
-        // suffix sums over digits (lanes 15 .. 0)
-        int suf = lane < 16 ? cnt : 0;
-#pragma unroll
-        for (int off = 1; off < 16; off <<= 1) {
-            const int y = __shfl_down_sync(0xffffffffu, suf, off);
-            if (lane + off < 16) suf += y;
-        }
-        const int above = suf - (lane < 16 ? cnt : 0);
-        const bool hit = lane < 16 && above < krem && above + cnt >= krem;
-        const unsigned hm = __ballot_sync(0xffffffffu, hit);
-        const int src = __ffs(hm) - 1;
-        const int a = __shfl_sync(0xffffffffu, above, src);
+        const int src = __ffs(__ballot_sync(0xffffffffu, bin >= 0)) - 1;
+        bin = __shfl_sync(0xffffffffu, bin, src);
+        krem = __shfl_sync(0xffffffffu, kr, src);
         cnt_sel = __shfl_sync(0xffffffffu, cnt, src);
-        prefix |= (uint32_t)src << shift;
-        mask |= 15u << shift;
-        krem -= a;
+        if (pass == 0) hi10 = (uint32_t)bin;
+        else *low = (hi10 << 10) | (uint32_t)bin;
+        __syncwarp();
     }
-    *low = prefix;
     *krem_out = krem;
     *cnt_out = cnt_sel;
 }
@@ -182,15 +195,30 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
     uint32_t T;
     int cnt_T;
     if (n1 <= kCandCap) {
-        // gather the threshold bin's keys; warp 0 resolves the low 20 bits
+        // gather the threshold bin's keys (one shared atomic per warp reserves
+        // the warp's slots); warp 0 then resolves the low 20 bits
+        int mine = 0;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) mine += (key[e] && (key[e] >> 20) == bin1);
+        const int lane = tid & 31;
+        int incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        int base = 0;
+        if (lane == 31 && incl > 0) base = atomicAdd(&s_ncand, incl);
+        base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
 #pragma unroll
         for (int e = 0; e < KPT; ++e)
-            if (key[e] && (key[e] >> 20) == bin1) cand[atomicAdd(&s_ncand, 1)] = key[e];
+            if (key[e] && (key[e] >> 20) == bin1) cand[base++] = key[e];
         __syncthreads();
         if (tid < 32) {
             uint32_t low;
             int kr, c;
-            warp_select20(cand, s_ncand, krem, &low, &kr, &c);
+            // the pass-1 histogram is no longer read: its first 1024 bins serve warp 0
+            warp_select20(cand, s_ncand, krem, hist, &low, &kr, &c);
             if (tid == 0) {
                 s_T = (bin1 << 20) | low;
                 s_krem = kr;
@@ -353,7 +381,7 @@ cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k,
     if (S <= 128 * 4) return launch_reg<4, 128>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 128 * 8) return launch_reg<8, 128>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 128 * 16) return launch_reg<16, 128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 128 * 32) return launch_reg<32, 128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 16) return launch_reg<16, 256>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 256 * 32) return launch_reg<32, 256>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 512 * 32) return launch_reg<32, 512>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 512 * 64) return launch_reg<64, 512>(scores, rows, Si, ki, idx, s, pdl);

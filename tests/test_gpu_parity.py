@@ -49,6 +49,7 @@ def run_full(loki, inp, dev, S=None, S_max=None, d=None, k=None, with_steps=Fals
         res["scores"] = loki.loki_score_lowdim(q_rot, Kt if Kt_lo is None else Kt_lo, S,
                                                d).cpu().numpy()
     torch.cuda.synchronize()
+    assert loki.loki_device_error(reset=True) == 0, "a staged kernel's bounded wait gave up"
     return res
 
 
@@ -193,6 +194,7 @@ def sampled_run(loki, dev, wl, n_rows, seed=7, plane=False):
     out = out.float().cpu().numpy()
     idx = idx.cpu().numpy()
     qh = q.float().cpu().numpy()
+    assert loki.loki_device_error(reset=True) == 0, "a staged kernel's bounded wait gave up"
     checks = []
     for b, h in rows:
         hk = h // wl.G
