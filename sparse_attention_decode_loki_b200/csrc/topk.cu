@@ -10,14 +10,15 @@
 // lowest indices first. All decisions are integer compares: the result is
 // exact and deterministic.
 //
-// Rows of up to 32768 keys (k_topk_reg): each thread holds a contiguous run of
-// keys in registers. One block pass histograms the top 12 key bits (4096
-// shared-memory bins: sign, exponent and 3 mantissa bits), which already
-// narrows the threshold to one bin holding a few percent of the row; those
-// keys are gathered and warp 0 resolves the remaining 20 bits alone with two
-// 10-bit passes over a warp-private histogram, so no further block barriers
-// are paid. (A bin too crowded
-// for the gather buffer -- heavy ties -- takes two 10-bit block passes.)
+// Rows of up to 32768 keys (k_topk_smem): keys in shared memory. One block
+// pass histograms the top 12 key bits (4096 shared-memory bins: sign,
+// exponent and 3 mantissa bits), which already narrows the threshold to one
+// bin holding a few percent of the row; those keys are gathered and warp 0
+// resolves the remaining 20 bits alone with two 10-bit passes over a
+// warp-private histogram, so no further block barriers are paid. (A bin too
+// crowded for the gather buffer -- heavy ties -- takes two 10-bit block
+// passes.) The compaction reads each thread's run of keys once into bit
+// masks and writes the selected indices in ascending order from them.
 // Longer rows (k_topk_long) keep keys in shared memory, or re-read them from
 // L2 when they do not fit, with 8-bit digits and warp-aggregated atomics.
 #include "common.cuh"
@@ -60,10 +61,34 @@ __device__ __forceinline__ int block_excl_scan(int v, int* buf, int* total) {
     return before;
 }
 
+// Within one chunk of 32 consecutive bins (base b0) of which the krem-th
+// largest counted key is known to lie in, find that bin with the whole warp:
+// lane l holds bin b0 + l, a suffix scan over lanes gives the keys above each
+// bin. Returns (bin, rank left inside it, its count) on every lane.
+__device__ __forceinline__ void warp_find_in_chunk(const uint32_t* h, int b0, int nb, int krem,
+                                                   int* bin, int* kr, int* cnt) {
+    const int lane = threadIdx.x & 31;
+    const int c = lane < nb ? (int)h[b0 + lane] : 0;
+    int suf = c;  // inclusive suffix sum over lanes (higher lanes = higher bins)
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, suf, off);
+        if (lane + off < 32) suf += y;
+    }
+    const int above = suf - c;
+    const unsigned hit = __ballot_sync(0xffffffffu, lane < nb && above < krem && above + c >= krem);
+    const int src = hit ? __ffs(hit) - 1 : 0;  // a hit always exists when the counts hold krem
+    *bin = b0 + src;
+    *kr = krem - __shfl_sync(0xffffffffu, above, src);
+    *cnt = __shfl_sync(0xffffffffu, c, src);
+}
+
 // Given per-bin counts in hist[0, nbins) (bins ordered by key), find the bin
 // holding the krem-th largest counted key. Thread t owns bins [t*per, (t+1)*per)
-// and reads them in a rotated order (bank-conflict free for per <= 32).
-// Writes the bin, the rank left inside it and the bin's count to shared memory.
+// (per <= 32, a power of two) and reads them in a rotated order (bank-conflict
+// free); the thread whose range holds the bin hands it to warp 0, which
+// searches the range in parallel. Writes the bin, the rank left inside it and
+// the bin's count to shared memory (valid after the function returns).
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int krem, int* buf,
                                          int* s_bin, int* s_krem, int* s_cnt) {
     const int per = nbins / (int)blockDim.x;
@@ -73,16 +98,20 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int kr
     for (int i = 0; i < per; ++i) local += (int)hist[b0 + ((i + rot) & (per - 1))];
     int total;
     const int before = block_excl_scan(local, buf, &total);
-    int above = total - before - local;  // keys in bins owned by higher threads
+    const int above = total - before - local;  // keys in bins owned by higher threads
     if (above < krem && above + local >= krem) {
-        for (int i = per - 1; i >= 0; --i) {
-            const int c = (int)hist[b0 + i];
-            if (above < krem && above + c >= krem) {
-                *s_bin = b0 + i;
-                *s_krem = krem - above;
-                *s_cnt = c;
-            }
-            above += c;
+        buf[0] = b0;
+        buf[1] = krem - above;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int bin, kr, cnt;
+        const int cb0 = min(max(buf[0], 0), nbins - per);  // stays inside hist whatever buf holds
+        warp_find_in_chunk(hist, cb0, per, buf[1], &bin, &kr, &cnt);
+        if (threadIdx.x == 0) {
+            *s_bin = bin;
+            *s_krem = kr;
+            *s_cnt = cnt;
         }
     }
     __syncthreads();
@@ -98,10 +127,10 @@ __device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int k
     const int lane = threadIdx.x & 31;
     uint32_t hi10 = 0u;
     int cnt_sel = 0;
-#pragma unroll
+#pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         const int shift = pass == 0 ? 10 : 0;
-#pragma unroll
+#pragma unroll 8
         for (int i = 0; i < 32; ++i) h[32 * i + lane] = 0u;
         __syncwarp();
         for (int i = lane; i < n; i += 32) {
@@ -110,7 +139,7 @@ __device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int k
         }
         __syncwarp();
         int local = 0;
-#pragma unroll
+#pragma unroll 8
         for (int i = 0; i < 32; ++i) local += (int)h[32 * lane + ((i + lane) & 31)];
         int suf = local;  // inclusive suffix sum over lanes
 #pragma unroll
@@ -118,23 +147,14 @@ __device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int k
             const int y = __shfl_down_sync(0xffffffffu, suf, off);
             if (lane + off < 32) suf += y;
         }
-        int above = suf - local;
-        int bin = -1, kr = 0, cnt = 0;
-        if (above < krem && above + local >= krem) {
-            for (int i = 31; i >= 0; --i) {
-                const int c = (int)h[32 * lane + i];
-                if (above < krem && above + c >= krem) {
-                    bin = 32 * lane + i;
-                    kr = krem - above;
-                    cnt = c;
-                }
-                above += c;
-            }
-        }
-        const int src = __ffs(__ballot_sync(0xffffffffu, bin >= 0)) - 1;
-        bin = __shfl_sync(0xffffffffu, bin, src);
-        krem = __shfl_sync(0xffffffffu, kr, src);
-        cnt_sel = __shfl_sync(0xffffffffu, cnt, src);
+        const int above = suf - local;
+        const unsigned hit = __ballot_sync(0xffffffffu, above < krem && above + local >= krem);
+        const int src = hit ? __ffs(hit) - 1 : 0;
+        int bin, kr, cnt;
+        warp_find_in_chunk(h, 32 * src, 32, krem - __shfl_sync(0xffffffffu, above, src), &bin, &kr,
+                           &cnt);
+        krem = kr;
+        cnt_sel = cnt;
         if (pass == 0) hi10 = (uint32_t)bin;
         else *low = (hi10 << 10) | (uint32_t)bin;
         __syncwarp();
@@ -143,49 +163,59 @@ __device__ __forceinline__ void warp_select20(const uint32_t* cand, int n, int k
     *cnt_out = cnt_sel;
 }
 
-template <int KPT, int NT>
-__global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ scores, int S, int k,
-                                                 int32_t* __restrict__ out) {
+// Rows of up to 32 * NT keys: keys in shared memory (zero-padded to a
+// multiple of 4; key 0 never comes from a score), every loop rolled and over
+// uint4 groups of 4 keys (a small kernel body that stays in the instruction
+// cache, and few instructions per key).
+template <int NT>
+__global__ void __launch_bounds__(NT) k_topk_smem(const float* __restrict__ scores, int S, int k,
+                                                  int32_t* __restrict__ out, int vec4) {
     constexpr int kCandCap = 2048;
-    __shared__ uint32_t hist[4096];
+    extern __shared__ uint4 keys4[];
+    __shared__ __align__(16) uint32_t hist[4096];
     __shared__ uint32_t cand[kCandCap];
     __shared__ int scan_buf[32];
     __shared__ int s_bin, s_krem, s_cnt, s_ncand;
     __shared__ uint32_t s_T;
-    const int tid = threadIdx.x;
+    const uint32_t* keys = reinterpret_cast<const uint32_t*>(keys4);
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int S4 = (S + 3) >> 2;
     const float* row = scores + (int64_t)blockIdx.x * S;
-    const int j0 = tid * KPT;
-    for (int i = tid; i < 4096; i += NT) hist[i] = 0u;
+#pragma unroll 1
+    for (int i = tid; i < 1024; i += NT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (tid == 0) s_ncand = 0;
     griddep_wait();  // scores come from the score kernel
     griddep_launch_dependents();
 
-    uint32_t key[KPT];
-    if ((S & 3) == 0) {
-#pragma unroll
-        for (int e = 0; e < KPT; e += 4) {
-            if (j0 + e < S) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(row + j0 + e));
-                key[e] = order_key(v.x);
-                key[e + 1] = order_key(v.y);
-                key[e + 2] = order_key(v.z);
-                key[e + 3] = order_key(v.w);
-            } else {
-                key[e] = key[e + 1] = key[e + 2] = key[e + 3] = 0u;
-            }
+    if (vec4) {  // S % 4 == 0 and scores 16-byte aligned
+        const float4* r4 = reinterpret_cast<const float4*>(row);
+#pragma unroll 1
+        for (int j = tid; j < S4; j += NT) {
+            const float4 v = __ldg(r4 + j);
+            keys4[j] = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
         }
     } else {
-#pragma unroll
-        for (int e = 0; e < KPT; ++e) key[e] = (j0 + e < S) ? order_key(__ldg(row + j0 + e)) : 0u;
+#pragma unroll 1
+        for (int j = tid; j < S4; j += NT) {
+            const int j4 = 4 * j;
+            keys4[j] = make_uint4(order_key(__ldg(row + j4)),
+                                  j4 + 1 < S ? order_key(__ldg(row + j4 + 1)) : 0u,
+                                  j4 + 2 < S ? order_key(__ldg(row + j4 + 2)) : 0u,
+                                  j4 + 3 < S ? order_key(__ldg(row + j4 + 3)) : 0u);
+        }
     }
-    // key 0 never comes from a score (NaN maps to the -inf key), so it marks
-    // padding: it is never counted, selected or histogrammed
     __syncthreads();
 
-    // pass 1: top 12 bits over the whole row
-#pragma unroll
-    for (int e = 0; e < KPT; ++e)
-        if (key[e]) atomicAdd(&hist[key[e] >> 20], 1u);
+    // pass 1: top 12 bits over the whole row (padding keys land in bin 0,
+    // below every real key, and never reach the threshold)
+#pragma unroll 1
+    for (int j = tid; j < S4; j += NT) {
+        const uint4 v = keys4[j];
+        atomicAdd(&hist[v.x >> 20], 1u);
+        atomicAdd(&hist[v.y >> 20], 1u);
+        atomicAdd(&hist[v.z >> 20], 1u);
+        atomicAdd(&hist[v.w >> 20], 1u);
+    }
     __syncthreads();
     find_bin(hist, 4096, k, scan_buf, &s_bin, &s_krem, &s_cnt);
     const uint32_t bin1 = (uint32_t)s_bin;
@@ -195,24 +225,31 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
     uint32_t T;
     int cnt_T;
     if (n1 <= kCandCap) {
-        // gather the threshold bin's keys (one shared atomic per warp reserves
-        // the warp's slots); warp 0 then resolves the low 20 bits
-        int mine = 0;
+        // gather the threshold bin's keys (one shared atomic per warp and
+        // step); warp 0 then resolves the low 20 bits
+        const int S4r = (S4 + 31) & ~31;
+#pragma unroll 1
+        for (int j = tid; j < S4r; j += NT) {
+            const uint4 v = j < S4 ? keys4[j] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+            const int mine = ((kk[0] >> 20) == bin1) + ((kk[1] >> 20) == bin1) +
+                             ((kk[2] >> 20) == bin1) + ((kk[3] >> 20) == bin1);
+            const unsigned any = __ballot_sync(0xffffffffu, mine > 0);
+            if (any) {
+                int incl = mine;
 #pragma unroll
-        for (int e = 0; e < KPT; ++e) mine += (key[e] && (key[e] >> 20) == bin1);
-        const int lane = tid & 31;
-        int incl = mine;
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += y;
+                }
+                int base = 0;
+                if (lane == 31) base = atomicAdd(&s_ncand, incl);
+                base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += y;
+                for (int e = 0; e < 4; ++e)
+                    if ((kk[e] >> 20) == bin1) cand[base++] = kk[e];
+            }
         }
-        int base = 0;
-        if (lane == 31 && incl > 0) base = atomicAdd(&s_ncand, incl);
-        base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
-#pragma unroll
-        for (int e = 0; e < KPT; ++e)
-            if (key[e] && (key[e] >> 20) == bin1) cand[base++] = key[e];
         __syncthreads();
         if (tid < 32) {
             uint32_t low;
@@ -232,21 +269,23 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
     } else {
         // a crowded bin (heavy ties): two more block passes of 10 bits each
         __syncthreads();
+#pragma unroll 1
         for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
         __syncthreads();
-#pragma unroll
-        for (int e = 0; e < KPT; ++e)
-            if (key[e] && (key[e] >> 20) == bin1) atomicAdd(&hist[(key[e] >> 10) & 1023u], 1u);
+#pragma unroll 1
+        for (int j = tid; j < 4 * S4; j += NT)
+            if ((keys[j] >> 20) == bin1) atomicAdd(&hist[(keys[j] >> 10) & 1023u], 1u);
         __syncthreads();
         find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem, &s_cnt);
         const uint32_t pre2 = (bin1 << 10) | (uint32_t)s_bin;
         krem = s_krem;
         __syncthreads();
+#pragma unroll 1
         for (int i = tid; i < 1024; i += NT) hist[i] = 0u;
         __syncthreads();
-#pragma unroll
-        for (int e = 0; e < KPT; ++e)
-            if (key[e] && (key[e] >> 10) == pre2) atomicAdd(&hist[key[e] & 1023u], 1u);
+#pragma unroll 1
+        for (int j = tid; j < 4 * S4; j += NT)
+            if ((keys[j] >> 10) == pre2) atomicAdd(&hist[keys[j] & 1023u], 1u);
         __syncthreads();
         find_bin(hist, 1024, krem, scan_buf, &s_bin, &s_krem, &s_cnt);
         T = (pre2 << 10) | (uint32_t)s_bin;
@@ -254,14 +293,28 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
         cnt_T = s_cnt;
     }
     // T is the k-th largest key; krem of the cnt_T keys equal to T are taken,
-    // lowest indices first
-
-    int gt = 0, eq = 0;
+    // lowest indices first. Thread t owns the q4 uint4 groups [t*q4, t*q4 + q4)
+    // (4*q4 <= 32 keys), read in a rotated order into bit masks.
+    const int q4 = (S4 + NT - 1) / NT;
+    const int g0 = tid * q4;
+    const int ng = max(0, min(q4, S4 - g0));
+    const bool pow2 = (q4 & (q4 - 1)) == 0;
+    uint32_t gtm = 0u, eqm = 0u;
+    const int nloop = pow2 ? q4 : ng;
+#pragma unroll 1
+    for (int i = 0; i < nloop; ++i) {
+        const int ii = pow2 ? ((i + tid) & (q4 - 1)) : i;
+        if (ii < ng) {
+            const uint4 v = keys4[g0 + ii];
+            const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-        gt += key[e] > T;
-        eq += key[e] == T;
+            for (int e = 0; e < 4; ++e) {
+                gtm |= (uint32_t)(kk[e] > T) << (4 * ii + e);
+                eqm |= (uint32_t)(kk[e] == T) << (4 * ii + e);
+            }
+        }
     }
+    const int gt = __popc(gtm), eq = __popc(eqm);
     int total, take_eq;
     if (krem == cnt_T) {
         take_eq = eq;  // every key equal to T is selected: no tie scan needed
@@ -270,19 +323,18 @@ __global__ void __launch_bounds__(NT) k_topk_reg(const float* __restrict__ score
         take_eq = max(0, min(eq, krem - eq_before));
     }
     int pos = block_excl_scan(gt + take_eq, scan_buf, &total);
+    // keys equal to T beyond the first take_eq (in index order) are dropped
+    uint32_t em = eqm;
+    for (int t = 0; t < take_eq; ++t) em &= em - 1u;
+    uint32_t take = gtm | (eqm & ~em);
     int32_t* o = out + (int64_t)blockIdx.x * k;
-    int eq_seen = 0;
-#pragma unroll
-    for (int e = 0; e < KPT; ++e) {
-        bool take = key[e] > T;
-        if (key[e] == T) {
-            take = eq_seen < take_eq;
-            ++eq_seen;
-        }
-        if (take) {
-            if (pos < k) o[pos] = j0 + e;  // pos < k by construction; the bound keeps writes in the row
-            ++pos;
-        }
+    const int j0 = 4 * g0;
+#pragma unroll 1
+    while (take) {
+        const int ii = __ffs(take) - 1;
+        take &= take - 1u;
+        if (pos < k) o[pos] = j0 + ii;  // pos < k by construction; the bound keeps writes in the row
+        ++pos;
     }
 }
 
@@ -367,24 +419,28 @@ __global__ void __launch_bounds__(512) k_topk_long(const float* __restrict__ sco
     }
 }
 
-template <int KPT, int NT>
-static cudaError_t launch_reg(const float* scores, int64_t rows, int S, int k, int32_t* idx,
+template <int NT>
+static cudaError_t launch_smem(const float* scores, int64_t rows, int S, int k, int32_t* idx,
                               cudaStream_t s, bool pdl) {
-    return launch_kernel(k_topk_reg<KPT, NT>, dim3((unsigned)rows), dim3(NT), 0, s, pdl, scores,
-                         S, k, idx);
+    const size_t smem = ((size_t)S + 3) / 4 * 16;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            k_topk_smem<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int vec4 = (S % 4 == 0) && (reinterpret_cast<uintptr_t>(scores) % 16 == 0);
+    return launch_kernel(k_topk_smem<NT>, dim3((unsigned)rows), dim3(NT), smem, s, pdl, scores, S,
+                         k, idx, vec4);
 }
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl) {
     const int Si = (int)S, ki = (int)k;
-    // find_bin needs 4096 and 1024 bins to split evenly over the threads (NT <= 1024)
-    if (S <= 128 * 4) return launch_reg<4, 128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 128 * 8) return launch_reg<8, 128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 128 * 16) return launch_reg<16, 128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 16) return launch_reg<16, 256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 32) return launch_reg<32, 256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 512 * 32) return launch_reg<32, 512>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 512 * 64) return launch_reg<64, 512>(scores, rows, Si, ki, idx, s, pdl);
+    // each thread owns at most 32 consecutive keys of the row
+    if (S <= 128 * 32) return launch_smem<128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 32) return launch_smem<256>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 512 * 32) return launch_smem<512>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 1024 * 32) return launch_smem<1024>(scores, rows, Si, ki, idx, s, pdl);
     {
         DevInfo di;
         cudaError_t e = dev_info(&di);
