@@ -68,6 +68,28 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (the job's timing is its slowest rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_step(max_rank_total_ms: float, steps: int, world: int) -> float:
+    """Each rank runs `steps` full layer-steps of its own replica in the timed region,
+    so the job completes steps * world layer-steps in the slowest rank's time."""
+    return max_rank_total_ms * 1e3 / (steps * world)
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Replicas draw independent inputs: rank r offsets the workload seed."""
+    return base_seed + 1_000_000 * rank
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -235,7 +257,7 @@ def build_gpu_inputs(wl, dev, rank):
 
     import sparse_attention_decode_loki_b200 as loki
     import workloads
-    wl_r = wl.with_(seed=wl.seed + 1_000_000 * rank) if rank else wl
+    wl_r = wl.with_(seed=replica_seed(wl.seed, rank))
     g = workloads.generate(wl_r)
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     K_cal = torch.from_numpy(g["K_cal"]).to(dev).to(dt)
@@ -345,13 +367,9 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     us_per_step_rank = total_ms * 1e3 / args.steps
-    value = us_per_step_rank / world
+    value = whole_job_us_per_step(total_ms, args.steps, world)
     nb = max(50, min(args.steps, 400))
     eager_us = statistics.mean(timed(decode, nb, 10)) * 1e3
 
@@ -406,11 +424,7 @@ def run_ours(args):
         idx_pin.copy_(idx, non_blocking=True)
 
     e2e_ms = timed(e2e_step, max(50, min(args.steps, 1000)), 5)
-    e2e_us = statistics.mean(e2e_ms) * 1e3
-    if world > 1:
-        t = torch.tensor([e2e_us], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_us = float(t.item())
+    e2e_us = max_over_ranks(statistics.mean(e2e_ms) * 1e3, world, dev)
     h2d = q_pin.numel() * q_pin.element_size()
     d2h = out_pin.numel() * out_pin.element_size() + idx_pin.numel() * idx_pin.element_size()
 
@@ -424,7 +438,7 @@ def run_ours(args):
     achieved = alg[dom] / (kern_us[dom] * 1e-6) / 1e9
     step_bytes = wl.loki_bytes()
     step_us = us_per_step_rank
-    prof_name = {"score_lowdim": "score_lowdim", "sparse_attention+combine": "sparse_attn"}[dom]
+    prof_name = {"score_lowdim": "score_plane", "sparse_attention+combine": "sparse_attn"}[dom]
     traffic = traffic_from_profiles(prof_name, wl.name)
 
     res = {

@@ -394,9 +394,17 @@ loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, i
     LOKI_PTR(q_rot, 16);
     LOKI_PTR(Kt_cache, 16);
     LOKI_PTR(scores, 4);
-    LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, 128, D,
-                                        d, scores, static_cast<cudaStream_t>(stream), false),
-              "loki_score_lowdim");
+    // a plane (row width < 128) goes through the same TMA-staged scan as the
+    // decode step; the rotated cache through the register-staged scan
+    if (D < 128)
+        LOKI_CUDA(loki::launch_score_plane(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, 128,
+                                           D, d, scores, static_cast<cudaStream_t>(stream), false),
+                  "loki_score_lowdim");
+    else
+        LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max,
+                                            128, D, d, scores, static_cast<cudaStream_t>(stream),
+                                            false),
+                  "loki_score_lowdim");
     return LOKI_OK;
 }
 
