@@ -318,26 +318,40 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
     float* scores = at<float>(ws, w.scores);
     int* done = at<int>(ws, w.done);
     const int rows = B * H_q;
-    // Four kernels: query projection (which also zeroes the attention
-    // kernel's row counters); score scan (over a low-dim key plane the
-    // TMA-staged scan, which starts streaming keys while the projection runs;
-    // over the row layout the register-staged scan); top-k; attention with
-    // its row merge. The first kernel is ordered normally after whatever
-    // precedes the call; the later ones use programmatic dependent launch.
-    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows), name);
-    if (Kt_lo != nullptr)
+    // Four kernels. Over a low-dim key plane: the TMA-staged score scan,
+    // which rotates the queries' first d_lo columns itself and streams keys
+    // at once, with the full query projection (which also zeroes the
+    // attention kernel's row counters) launched beside it; over the row
+    // layout: the projection, then the register-staged scan. Then top-k and
+    // attention with its row merge. The first kernel is ordered normally
+    // after whatever precedes the call; the second and top-k use programmatic
+    // dependent launch.
+    const bool fused = Kt_lo != nullptr && loki::score_plane_fuses(t, H_q / H_kv, d_lo, D);
+    if (fused) {
         LOKI_CUDA(loki::launch_score_plane(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
-                                           scores, s, true),
+                                           scores, s, false, q, P),
                   name);
-    else
-        LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, D, d,
-                                            scores, s, true),
+        LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows, true),
                   name);
+    } else {
+        LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows),
+                  name);
+        if (Kt_lo != nullptr)
+            LOKI_CUDA(loki::launch_score_plane(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo,
+                                               d, scores, s, true),
+                      name);
+        else
+            LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, D,
+                                                d, scores, s, true),
+                      name);
+    }
     LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
+    // attention is ordered normally after top-k (no early launch): its CTAs
+    // then start on drained SMs that take its large-L1 split
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
-                                            true),
+                                            false),
               name);
     return LOKI_OK;
 }

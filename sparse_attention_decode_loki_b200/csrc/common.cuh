@@ -88,12 +88,24 @@ struct Split {
     int64_t per;
 };
 
+// Sets the preferred L1/shared-memory split of `func` (percent of the
+// maximum shared memory, or cudaSharedmemCarveoutMaxL1/MaxShared) once per
+// device; the first request for a kernel wins. An SM changes its split only
+// when it is empty, so kernels meant to be resident side by side (a
+// programmatic dependent launched early next to its predecessor) ask for the
+// same, largest, shared split; register-gather kernels, whose loads in flight
+// land in L1, ask for the largest L1 and are launched onto drained SMs.
+cudaError_t prefer_carveout(const void* func, int carveout);
+
 // Launch `kern` on `s`; with pdl the launch carries the programmatic
 // stream-serialization attribute (the kernel must griddep_wait() before
 // reading anything its predecessor writes).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                  cudaStream_t s, bool pdl, Args... args) {
+    const cudaError_t ec =
+        prefer_carveout(reinterpret_cast<const void*>(kern), cudaSharedmemCarveoutMaxShared);
+    if (ec != cudaSuccess) return ec;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

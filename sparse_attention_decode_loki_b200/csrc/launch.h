@@ -28,10 +28,13 @@ int* device_error_word();
 void set_last_error(const char* msg);
 
 // ---- decode steps --------------------------------------------------------
-// also zeroes done[0, n_done) when done is not null
+// also zeroes done[0, n_done) when done is not null. With pdl it is launched
+// as a programmatic dependent of the preceding kernel (the score scan that
+// rotates its own queries) and runs beside it; it then completes only after
+// that kernel does.
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
                                  int D, float* q_rot, cudaStream_t s, int* done = nullptr,
-                                 int n_done = 0);
+                                 int n_done = 0, bool pdl = false);
 
 // `row` is the row length (and stride) of the key buffer scanned: D for the
 // rotated cache, d_lo for a low-dimensional key plane.
@@ -39,12 +42,18 @@ cudaError_t launch_score_lowdim(Dt dt, const float* q_rot, const void* Kt, int B
                                 int H_kv, int64_t S, int64_t S_max, int D, int row, int d,
                                 float* scores, cudaStream_t s, bool pdl);
 
+// Whether launch_score_plane can rotate the queries itself for this shape.
+bool score_plane_fuses(Dt dt, int G, int d_lo, int D);
+
 // TMA-staged scan of a low-dim key plane Klo [B, H_kv, S_max, d_lo]. With pdl
-// it may start while the projection that writes q_rot is still running (it
-// streams keys first, then waits).
+// it may start while the projection that writes q_rot is still running: it
+// streams keys first and its consumers wait for q_rot. Given the raw queries
+// q and the bases P (head dim 128; score_plane_fuses) the consumers rotate the
+// query themselves, and the scan is launched without pdl whatever pdl says.
 cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
                                int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
-                               float* scores, cudaStream_t s, bool pdl);
+                               float* scores, cudaStream_t s, bool pdl, const void* q = nullptr,
+                               const float* P = nullptr);
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl);

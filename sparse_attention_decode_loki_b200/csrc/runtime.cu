@@ -3,7 +3,9 @@
 // (SM count x resident CTAs per SM) so every CTA of a persistent split runs in
 // a single wave.
 #include <mutex>
+#include <set>
 #include <unordered_map>
+#include <utility>
 
 #include "launch.h"
 
@@ -35,7 +37,20 @@ struct OccHash {
     }
 };
 std::unordered_map<OccKey, int, OccHash> g_occ;
+std::set<std::pair<int, const void*>> g_carveout_set;
 }  // namespace
+
+cudaError_t prefer_carveout(const void* func, int carveout) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_carveout_set.count({dev, func})) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
+    if (e != cudaSuccess) return e;
+    g_carveout_set.insert({dev, func});
+    return cudaSuccess;
+}
 
 cudaError_t dev_info(DevInfo* out) {
     int dev = 0;

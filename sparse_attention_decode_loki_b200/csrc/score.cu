@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(256) k_project_query(const typename E::T* __re
                                                        const float* __restrict__ P,
                                                        float* __restrict__ q_rot, int B, int H_q,
                                                        int G, int D, int* __restrict__ done,
-                                                       int n_done) {
+                                                       int n_done, int hold) {
     __shared__ float Ps[128][kProjCols];
     __shared__ float qs[kProjRows][128];
     // the next kernel (the score scan) may start streaming keys right away
@@ -91,6 +91,11 @@ __global__ void __launch_bounds__(256) k_project_query(const typename E::T* __re
         const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
         if (c0 + lane < D) q_rot[row * D + c0 + lane] = acc;
     }
+    // hold: launched beside the score scan, this grid completes only after the
+    // scan does (one waiting thread is enough), so the kernels that wait on
+    // it also see the scan's scores
+    if (hold && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        griddep_wait();
 }
 
 template <class E, int G>
@@ -169,16 +174,18 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
 }
 
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
-                                 int D, float* q_rot, cudaStream_t s, int* done, int n_done) {
+                                 int D, float* q_rot, cudaStream_t s, int* done, int n_done,
+                                 bool pdl) {
     const int G = H_q / H_kv;
     dim3 grid(H_kv, (D + kProjCols - 1) / kProjCols, (B * G + kProjRows - 1) / kProjRows);
+    const int hold = pdl ? 1 : 0;
     if (dt == kF32)
-        k_project_query<ElemF32><<<grid, 256, 0, s>>>(static_cast<const float*>(q), P, q_rot, B,
-                                                      H_q, G, D, done, n_done);
-    else
-        k_project_query<ElemBF16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), P,
-                                                       q_rot, B, H_q, G, D, done, n_done);
-    return cudaGetLastError();
+        return launch_kernel(k_project_query<ElemF32>, grid, dim3(256), 0, s, pdl,
+                             static_cast<const float*>(q), P, q_rot, B, H_q, G, D, done, n_done,
+                             hold);
+    return launch_kernel(k_project_query<ElemBF16>, grid, dim3(256), 0, s, pdl,
+                         static_cast<const __nv_bfloat16*>(q), P, q_rot, B, H_q, G, D, done,
+                         n_done, hold);
 }
 
 template <class E, int G>

@@ -13,9 +13,11 @@
 // of every tile for all G query heads of the unit (whole row per thread: no
 // shuffles, coalesced score stores), reading the row's 16-byte chunks in a
 // rotated order so a quarter-warp touches distinct banks. The ring keeps up
-// to ~90 KB per SM in flight without holding it in registers. Launched right behind the query
-// projection (programmatic dependent launch): the producer starts streaming
-// keys at once, and only the consumers wait for the projection's q~.
+// to ~90 KB per SM in flight without holding it in registers. In the decode
+// call the scan comes first and rotates the queries itself (the full query
+// projection runs beside it); as a step of its own it reads q~ and may be
+// launched right behind the projection (programmatic dependent launch): the
+// producer then starts streaming keys at once, and only the consumers wait.
 #include "common.cuh"
 #include "launch.h"
 #include "tma.cuh"
@@ -32,9 +34,17 @@ constexpr int kScoreMaxStages = 16;
 
 // NV = 16-byte chunks per plane row (d_lo * elem / 16). A tile is 256 rows,
 // one per consumer thread; stages = ring bytes / tile bytes.
-template <class E, int G, int NV>
+//
+// kFuseQ: the consumers rotate the query themselves, q~[:d] = q P[:, :d], per
+// (batch, KV head) unit, from q and P (head dim 128), so the scan needs no
+// projection kernel before it: thread (part p, column c) keeps the 128 /
+// parts rows of column c of P that it needs in registers, prefetched one unit
+// ahead, and the per-part partial sums meet in shared memory. Without it the
+// consumers read q~ from q_rot after the preceding kernel completes.
+template <class E, int G, int NV, bool kFuseQ>
 __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
-    const float* __restrict__ q_rot, const typename E::T* __restrict__ Klo,
+    const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
+    const float* __restrict__ P, const typename E::T* __restrict__ Klo,
     float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
     int D, int d, int64_t total, int64_t per) {
     constexpr int KV = E::kVec;
@@ -44,8 +54,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
     constexpr int kStages = (kScoreRingBytes / kTile) < kScoreMaxStages ? (kScoreRingBytes / kTile)
                                                                       : kScoreMaxStages;
     static_assert(kStages >= 2, "ring too small");
+    constexpr int C = NV * KV;                     // plane row width in elements
+    constexpr int kParts = kScoreConsumers / C;    // row blocks of P
+    constexpr int kR = 128 / kParts;               // rows of P per thread
+    constexpr int QN = (G * 128 + kScoreConsumers - 1) / kScoreConsumers;
     extern __shared__ __align__(128) unsigned char ring[];
     __shared__ uint64_t full[kStages], empty[kStages];
+    __shared__ float s_q[kFuseQ ? G * 128 : 1];
+    __shared__ float s_part[kFuseQ ? kParts * G * C : 1];
+    __shared__ float s_qlo[kFuseQ ? G * C : 1];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -93,12 +110,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
     }
 
     // ---------------- consumers: one row of each tile per thread ----------------
-    // q~ comes from the projection kernel, which may still be running: the
-    // producer above streams keys without waiting, the consumers wait here.
-    griddep_wait();
+    // Unfused, q~ comes from the projection kernel, which may still be
+    // running: the producer above streams keys without waiting, the consumers
+    // wait here.
+    if constexpr (!kFuseQ) griddep_wait();
     // chunk c of a row is read at rotation (c + tid / 2) % NV: the 8 threads
     // of a quarter-warp then hit 8 distinct 16-byte bank groups
     const int rot = (tid >> 1) & (NV - 1);
+    const int pc = tid % C, pp = tid / C;  // fused rotation: column and row block of P
+    float pf[kFuseQ ? kR : 1], qf[kFuseQ ? QN : 1];
+    // loads P[hk][pp*kR + j][pc] (zero beyond column d) and the unit's G query rows
+#define LOKI_FETCH_UNIT(unit_)                                                              \
+    {                                                                                      \
+        const int fb = (int)((unit_) / H_kv), fh = (int)((unit_) % H_kv);                  \
+        const float* Pp = P + ((int64_t)fh * 128 + pp * kR) * 128 + pc;                    \
+        _Pragma("unroll") for (int j = 0; j < kR; ++j) pf[j] =                            \
+            pc < d ? __ldg(Pp + j * 128) : 0.f;                                            \
+        const typename E::T* qb = q + ((int64_t)fb * H_q + (int64_t)fh * G) * 128;         \
+        _Pragma("unroll") for (int e = 0; e < QN; ++e) {                                   \
+            const int qi = tid + e * kScoreConsumers;                                      \
+            qf[e] = qi < G * 128 ? E::load1(qb + qi) : 0.f;                                \
+        }                                                                                  \
+    }
+    if constexpr (kFuseQ)
+        if (R0 < R1) LOKI_FETCH_UNIT(R0 / S)
     bool bad = false;
     int i = 0;
     for (int64_t r = R0; r < R1;) {
@@ -110,15 +145,50 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
         // qv holds q~ in this thread's rotated chunk order: slot cc holds
         // chunk (cc + rot) % NV, so the row loop indexes registers statically
         float qv[G][NV * KV];
+        if constexpr (kFuseQ) {
+            named_sync(1, kScoreConsumers);  // the previous unit's readers are done
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+            for (int e = 0; e < QN; ++e) {
+                const int qi = tid + e * kScoreConsumers;
+                if (qi < G * 128) s_q[qi] = qf[e];
+            }
+            named_sync(1, kScoreConsumers);
 #pragma unroll
-            for (int cc = 0; cc < NV; ++cc)
+            for (int g = 0; g < G; ++g) {
+                float a = 0.f;
 #pragma unroll
-                for (int e = 0; e < KV; ++e) {
-                    const int col = ((cc + rot) & (NV - 1)) * KV + e;
-                    qv[g][cc * KV + e] = col < d ? __ldg(q_rot + (qrow0 + g) * D + col) : 0.f;
-                }
+                for (int j = 0; j < kR; ++j) a = fmaf(s_q[g * 128 + pp * kR + j], pf[j], a);
+                s_part[(pp * G + g) * C + pc] = a;
+            }
+            named_sync(1, kScoreConsumers);
+            for (int x = tid; x < G * C; x += kScoreConsumers) {
+                float a = 0.f;
+#pragma unroll 4
+                for (int p2 = 0; p2 < kParts; ++p2) a += s_part[p2 * G * C + x];
+                s_qlo[x] = a;
+            }
+            named_sync(1, kScoreConsumers);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int cc = 0; cc < NV; ++cc)
+#pragma unroll
+                    for (int e = 0; e < KV; ++e)
+                        qv[g][cc * KV + e] = s_qlo[g * C + ((cc + rot) & (NV - 1)) * KV + e];
+            // the next unit's P block and queries load behind this unit's tiles
+            if ((unit + 1) * S < R1) LOKI_FETCH_UNIT(unit + 1)
+        } else {
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int cc = 0; cc < NV; ++cc)
+#pragma unroll
+                    for (int e = 0; e < KV; ++e) {
+                        const int col = ((cc + rot) & (NV - 1)) * KV + e;
+                        qv[g][cc * KV + e] = col < d ? __ldg(q_rot + (qrow0 + g) * D + col) : 0.f;
+                    }
+        }
+#undef LOKI_FETCH_UNIT
 
         float* srow = scores + qrow0 * S + s0;
         for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
@@ -154,17 +224,28 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
     }
 }
 
-template <class E, int G, int NV>
-static cudaError_t plane_impl(const float* q_rot, const void* Klo, float* scores, int* err, int B,
-                              int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
-                              cudaStream_t s, bool pdl) {
+// Arguments shared by every instantiation of the launch path.
+struct PlaneArgs {
+    const float* q_rot;  // q~ rows (unfused), or
+    const void* q;       // raw queries and
+    const float* P;      // the PCA bases (fused)
+    const void* Klo;
+    float* scores;
+    int* err;
+    int B, H_q, H_kv;
+    int64_t S, S_max;
+    int D, d;
+};
+
+template <class E, int G, int NV, bool kFuseQ>
+static cudaError_t plane_impl(const PlaneArgs& a, cudaStream_t s, bool pdl) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     constexpr int kTile = kScoreConsumers * NV * 16;
     constexpr int kStages = (kScoreRingBytes / kTile) < kScoreMaxStages ? (kScoreRingBytes / kTile)
                                                                       : kScoreMaxStages;
-    auto kern = k_score_plane<E, G, NV>;
+    auto kern = k_score_plane<E, G, NV, kFuseQ>;
     const size_t smem = (size_t)kStages * kTile;
     static bool attr_set[64] = {};
     if (di.device < 64 && !attr_set[di.device]) {
@@ -172,49 +253,45 @@ static cudaError_t plane_impl(const float* q_rot, const void* Klo, float* scores
         if (e != cudaSuccess) return e;
         attr_set[di.device] = true;
     }
-    const int64_t total = (int64_t)B * H_kv * S;
+    const int64_t total = (int64_t)a.B * a.H_kv * a.S;
     const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, kScoreThreads, smem);
     int64_t grid = (total + kScoreConsumers - 1) / kScoreConsumers;
     if (grid > resident) grid = resident;
     const int64_t per = (total + grid - 1) / grid;
     grid = (total + per - 1) / per;
     using T = typename E::T;
-    return launch_kernel(kern, dim3((unsigned)grid), dim3(kScoreThreads), smem, s, pdl, q_rot,
-                         static_cast<const T*>(Klo), scores, err, H_q, H_kv, (int)S, S_max, D, d,
-                         total, per);
+    return launch_kernel(kern, dim3((unsigned)grid), dim3(kScoreThreads), smem, s, pdl, a.q_rot,
+                         static_cast<const T*>(a.q), a.P, static_cast<const T*>(a.Klo), a.scores,
+                         a.err, a.H_q, a.H_kv, (int)a.S, a.S_max, a.D, a.d, total, per);
 }
 
 template <class E, int G, int NV>
-static cudaError_t plane_if(const float* q_rot, const void* Klo, float* scores, int* err, int B,
-                            int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
-                            cudaStream_t s, bool pdl) {
-    if constexpr (G * NV * E::kVec <= 64)
-        return plane_impl<E, G, NV>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
-    else
+static cudaError_t plane_if(const PlaneArgs& a, cudaStream_t s, bool pdl) {
+    if constexpr (G * NV * E::kVec <= 64) {
+        if (a.q != nullptr) return plane_impl<E, G, NV, true>(a, s, pdl);
+        return plane_impl<E, G, NV, false>(a, s, pdl);
+    } else {
         return cudaErrorInvalidValue;  // not dispatched (see score_plane_supported)
+    }
 }
 
 template <class E, int G>
-static cudaError_t plane_nv(int nv, const float* q_rot, const void* Klo, float* scores, int* err,
-                            int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
-                            cudaStream_t s, bool pdl) {
+static cudaError_t plane_nv(int nv, const PlaneArgs& a, cudaStream_t s, bool pdl) {
     switch (nv) {
-        case 1: return plane_if<E, G, 1>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
-        case 2: return plane_if<E, G, 2>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
-        case 4: return plane_if<E, G, 4>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
-        case 8: return plane_if<E, G, 8>(q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+        case 1: return plane_if<E, G, 1>(a, s, pdl);
+        case 2: return plane_if<E, G, 2>(a, s, pdl);
+        case 4: return plane_if<E, G, 4>(a, s, pdl);
+        case 8: return plane_if<E, G, 8>(a, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
 
 template <class E>
-static cudaError_t plane_dispatch(int G, int nv, const float* q_rot, const void* Klo,
-                                  float* scores, int* err, int B, int H_q, int H_kv, int64_t S,
-                                  int64_t S_max, int D, int d, cudaStream_t s, bool pdl) {
+static cudaError_t plane_dispatch(int G, int nv, const PlaneArgs& a, cudaStream_t s, bool pdl) {
     switch (G) {
-#define LOKI_G(g)                                                                              \
-    case g:                                                                                    \
-        return plane_nv<E, g>(nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d, s, pdl);
+#define LOKI_G(g) \
+    case g:       \
+        return plane_nv<E, g>(nv, a, s, pdl);
         LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
 #undef LOKI_G
         default: return cudaErrorInvalidValue;
@@ -230,21 +307,33 @@ bool score_plane_supported(Dt dt, int G, int d_lo) {
     return row_bytes % 16 == 0 && (nv == 1 || nv == 2 || nv == 4 || nv == 8) && G * nv * kv <= 64;
 }
 
+bool score_plane_fuses(Dt dt, int G, int d_lo, int D) {
+    return D == 128 && score_plane_supported(dt, G, d_lo);
+}
+
 cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
                                int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
-                               float* scores, cudaStream_t s, bool pdl) {
+                               float* scores, cudaStream_t s, bool pdl, const void* q,
+                               const float* P) {
     int* err = device_error_word();
     if (err == nullptr) return cudaErrorInvalidDevice;
     const int G = H_q / H_kv;
-    if (!score_plane_supported(dt, G, d_lo))
+    if (!score_plane_supported(dt, G, d_lo)) {
+        // the register-staged scan reads q~ from q_rot: it cannot rotate
+        if (q != nullptr) return cudaErrorInvalidValue;
         return launch_score_lowdim(dt, q_rot, Klo, B, H_q, H_kv, S, S_max, D, d_lo, d, scores, s,
                                    pdl);
+    }
     const int nv = d_lo * (dt == kF32 ? 4 : 2) / 16;
-    if (dt == kF32)
-        return plane_dispatch<ElemF32>(G, nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D,
-                                       d, s, pdl);
-    return plane_dispatch<ElemBF16>(G, nv, q_rot, Klo, scores, err, B, H_q, H_kv, S, S_max, D, d,
-                                    s, pdl);
+    const bool fuse = q != nullptr && P != nullptr;
+    if (fuse && D != 128) return cudaErrorInvalidValue;  // the fused rotation takes head dim 128
+    // a scan that rotates its own queries reads q at once: it is ordered
+    // normally after the preceding work, never launched early beside it
+    if (fuse) pdl = false;
+    const PlaneArgs a{q_rot, fuse ? q : nullptr, fuse ? P : nullptr, Klo, scores, err, B, H_q,
+                      H_kv, S, S_max, D, d};
+    if (dt == kF32) return plane_dispatch<ElemF32>(G, nv, a, s, pdl);
+    return plane_dispatch<ElemBF16>(G, nv, a, s, pdl);
 }
 
 }  // namespace loki

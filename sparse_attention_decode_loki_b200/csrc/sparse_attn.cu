@@ -3,39 +3,51 @@
 // "Visual Insights" Figure 1 caption: the full-dimensional keys give the
 // final attention scores).
 //
-// One warp per (row, chunk of the selected list); no block barriers. The warp
-// stages its selected indices in shared memory, then each row group of lanes
-// (16 lanes for bf16, 32 for fp32) gathers one 256/512-byte key row and the
-// matching value row per step, 8 rows in flight; every row is a random but
-// contiguous gather. Scores use all D dimensions in fp32; the softmax runs
-// online in base 2 with the scale folded into q~. The warp merges its row
-// groups with shuffles and writes one partial; the last warp to finish a row
-// (a per-row atomic counter) merges that row's partials into the output, so
-// no separate combine kernel runs.
+// Every warp of one wave owns an equal run of 16-key blocks of the selected
+// lists (rows laid end to end); no block barriers. The warp stages its
+// selected indices in shared memory, then each row group of lanes (16 lanes
+// for bf16, 32 for fp32) gathers one 256/512-byte key row and the matching
+// value row per step, 8 rows in flight; every row is a random but contiguous
+// gather. Scores use all D dimensions in fp32; the softmax runs online in
+// base 2 with the scale folded into q~. The warp merges its row groups with
+// shuffles and, per row it touches, writes the output (a whole row) or one
+// partial; the last warp to finish a row (a per-row atomic counter) merges
+// that row's partials into the output, so no separate combine kernel runs.
 #include "common.cuh"
 #include "launch.h"
 
 namespace loki {
 
 // Work decomposition. Each (batch, query head) row's k selected positions are
-// cut into nchunk chunks; a work item is one (row, chunk) and one warp owns one
-// item at a time (grid-stride over items). nchunk is chosen so the items fill
-// one wave of resident warps. Partials of row r sit in slots [r*nchunk, ...).
-constexpr int kMinChunk = 16;
+// cut into blocks of kBlk; the rows' blocks are laid end to end (N in all)
+// and every warp of one full wave takes an equal contiguous range of them,
+// warp w the blocks [w N / W, (w + 1) N / W). A range covers the tail of one
+// row, whole rows and the head of another, so every SM gets the same share of
+// the gather. A warp that covers a whole row writes its output directly;
+// otherwise it leaves a partial (m, l, acc) for each row it touches. The
+// warps touching row r are consecutive, w_first(r) .. w_last(r), and warp w's
+// partial of row r goes to slot r + w: no two (row, warp) pairs share a slot
+// since a later warp never touches an earlier row. Slots stay below rows + W.
+constexpr int kBlk = 16;
 constexpr int kWarpIdx = 256;  // indices staged per warp per step
 
 int64_t sparse_max_parts(int64_t rows, int64_t k) {
     int64_t cap = 10240 / rows;
     if (cap < 1) cap = 1;
-    const int64_t by_k = (k + kMinChunk - 1) / kMinChunk;
+    const int64_t by_k = (k + kBlk - 1) / kBlk;
     return (by_k < cap ? by_k : cap) + 2;
+}
+
+// The warp whose block range holds block b (W warps over N blocks).
+__device__ __forceinline__ int64_t owner_warp(int64_t b, int64_t W, int64_t N) {
+    return ((b + 1) * W - 1) / N;
 }
 
 template <class E>
 __global__ void __launch_bounds__(256) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
-    int64_t S_max, int k, float scale_log2, int chunk, int nchunk, int64_t n_items,
+    int64_t S_max, int k, float scale_log2, int nblk, int64_t N, int64_t W,
     float2* __restrict__ part_ml, float* __restrict__ part_acc, int* __restrict__ done,
     typename E::T* __restrict__ out) {
     constexpr int D = 128;
@@ -53,12 +65,16 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
     griddep_wait();  // q_rot and the selected indices come from earlier kernels
     griddep_launch_dependents();
 
-    const int64_t nwarps = (int64_t)gridDim.x * 8;
-    for (int64_t item = (int64_t)blockIdx.x * 8 + warp; item < n_items; item += nwarps) {
-        const int64_t r = item / nchunk;
-        const int c = (int)(item - r * nchunk);
-        const int j0 = c * chunk;
-        const int j1 = min(k, j0 + chunk);
+    // this warp's blocks [bcur, bend); W <= N, so no warp's range is empty
+    const int64_t w = (int64_t)blockIdx.x * 8 + warp;
+    int64_t bcur = w < W ? w * N / W : 0;
+    const int64_t bend = w < W ? (w + 1) * N / W : 0;
+    while (bcur < bend) {
+        const int64_t r = bcur / nblk;
+        const int64_t rb1 = min64(bend, (r + 1) * nblk);
+        const int j0 = (int)(bcur - r * nblk) * kBlk;
+        const int j1 = min(k, (int)(rb1 - r * nblk) * kBlk);
+        bcur = rb1;
         const int b = (int)(r / H_q), h = (int)(r % H_q);
         const int64_t unit = (int64_t)b * H_kv + h / G;
 
@@ -146,35 +162,48 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
             }
             m = M;
         }
+        const int64_t wf = owner_warp(r * nblk, W, N);
+        const int64_t wl = owner_warp((r + 1) * nblk - 1, W, N);
+        if (wf == wl) {  // the whole row is this warp's: normalise and write it
+            if (grp == 0) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                for (int e = 0; e < KV; ++e) out[r * D + sub * KV + e] = E::from_float(acc[e] * inv);
+            }
+            continue;
+        }
+        const int64_t slot = r + w;
         if (grp == 0) {
-            float* pa = part_acc + item * D + sub * KV;
+            float* pa = part_acc + slot * D + sub * KV;
 #pragma unroll
             for (int e = 0; e < KV; e += 4)
                 *reinterpret_cast<float4*>(pa + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-            if (sub == 0) part_ml[item] = make_float2(m, l);
+            if (sub == 0) part_ml[slot] = make_float2(m, l);
         }
-        // The last warp to finish a chunk of row r merges the row's partials
+        // The last warp to finish its part of row r merges the row's partials
         // (its own included) into out[r]: publish, count, and only the warp
-        // that sees the count reach nchunk reads the others' partials.
+        // that sees the count reach the number of parts reads the others'.
+        const int nparts = (int)(wl - wf + 1);
         __threadfence();  // each lane's partial writes are visible device-wide...
-        __syncwarp();     // ...before lane 0 counts the chunk as done
+        __syncwarp();     // ...before lane 0 counts the part as done
         int prev = 0;
         if (lane == 0) prev = atomicAdd(done + r, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev == nchunk - 1) {
+        if (prev == nparts - 1) {
             __threadfence();
-            const float2* ml = part_ml + r * nchunk;
+            const float2* ml = part_ml + r + wf;
+            const float* pacc = part_acc + (r + wf) * D;
             float M = -INFINITY;
-            for (int p = 0; p < nchunk; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
+            for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
             float Lsum = 0.f, A[D / 32];
 #pragma unroll
             for (int e = 0; e < D / 32; ++e) A[e] = 0.f;
             if (M != -INFINITY) {
-                for (int p = 0; p < nchunk; ++p) {
+                for (int p = 0; p < nparts; ++p) {
                     const float2 mlp = __ldcg(&ml[p]);
                     const float sc = exp2f(mlp.x - M);
                     Lsum += mlp.y * sc;
-                    const float* pa = part_acc + (r * nchunk + p) * D;
+                    const float* pa = pacc + (int64_t)p * D;
 #pragma unroll
                     for (int e = 0; e < D / 32; ++e) A[e] += __ldcg(pa + e * 32 + lane) * sc;
                 }
@@ -198,23 +227,25 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)B * H_q;
     auto kern = k_sparse_attn<E>;
-    const int64_t warps = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0) * 8;
-    int64_t nchunk = warps / rows;
-    if (nchunk < 1) nchunk = 1;
-    const int64_t cap = sparse_max_parts(rows, k);
-    if (nchunk > cap) nchunk = cap;
-    int64_t chunk = (k + nchunk - 1) / nchunk;
-    chunk = (chunk + kMinChunk - 1) / kMinChunk * kMinChunk;
-    nchunk = (k + chunk - 1) / chunk;
-    const int64_t n_items = rows * nchunk;
-    int64_t grid = (n_items + 7) / 8;
-    const int64_t max_grid = warps / 8;
-    if (grid > max_grid) grid = max_grid;
+    // the gathers in flight live in L1: the smallest shared split that still
+    // holds two CTAs' staged indices (8 KB each, plus 1 KB reserved per CTA)
+    const int pct = (2 * (8 + 1) * 1024 * 100 + di.smem_optin - 1) / di.smem_optin + 1;
+    e = prefer_carveout((const void*)kern, pct);
+    if (e != cudaSuccess) return e;
+    const int64_t nblk = (k + kBlk - 1) / kBlk;
+    const int64_t N = rows * nblk;
+    // one full wave of warps, but no more warps than blocks (no empty range)
+    // and no more partial slots (rows + W) than the workspace holds
+    int64_t W = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0) * 8;
+    const int64_t cap = rows * (sparse_max_parts(rows, k) - 1);
+    if (W > cap) W = cap;
+    if (W > N) W = N;
+    const int64_t grid = (W + 7) / 8;
     using T = typename E::T;
     return launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
                          static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv,
-                         (int)S, S_max, (int)k, scale * kLog2e, (int)chunk, (int)nchunk, n_items,
-                         part_ml, part_acc, done, static_cast<T*>(out));
+                         (int)S, S_max, (int)k, scale * kLog2e, (int)nblk, N, W, part_ml,
+                         part_acc, done, static_cast<T*>(out));
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,

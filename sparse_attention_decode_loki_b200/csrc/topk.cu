@@ -188,11 +188,25 @@ __global__ void __launch_bounds__(NT) k_topk_smem(const float* __restrict__ scor
     griddep_launch_dependents();
 
     if (vec4) {  // S % 4 == 0 and scores 16-byte aligned
+        // 8 loads in flight per thread before any is used: the row arrives in
+        // one or two memory round trips instead of one per group
+        constexpr int kInFlight = 8;
         const float4* r4 = reinterpret_cast<const float4*>(row);
 #pragma unroll 1
-        for (int j = tid; j < S4; j += NT) {
-            const float4 v = __ldg(r4 + j);
-            keys4[j] = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
+        for (int j0 = tid; j0 < S4; j0 += kInFlight * NT) {
+            float4 v[kInFlight];
+#pragma unroll
+            for (int u = 0; u < kInFlight; ++u) {
+                const int j = j0 + u * NT;
+                v[u] = j < S4 ? __ldg(r4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kInFlight; ++u) {
+                const int j = j0 + u * NT;
+                if (j < S4)
+                    keys4[j] = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z),
+                                          order_key(v[u].w));
+            }
         }
     } else {
 #pragma unroll 1
