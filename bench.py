@@ -389,8 +389,51 @@ def run_ours(args):
                                                                        wl.scale, out, sp_ws),
     }
     # (the decode call fuses the rotation into the score kernel and the merge
-    # into the attention kernel; the step entry points time them separately)
-    kern_us = {n_: statistics.mean(timed(f_, nb, 10)) * 1e3 for n_, f_ in comps.items()}
+    # into the attention kernel; the step entry points time them separately).
+    # Device time of one call with a cold L2, without the per-replay launch
+    # overhead of a graph: one graph holds R x (L2 flush, call), another R x
+    # (L2 flush); the difference of their CUDA-event times over R is the
+    # call's time, its launch gaps inside a graph included.
+    def diff_us(fn, R=8, reps=5):
+        fn()
+        torch.cuda.synchronize()
+
+        def capture(body):
+            g_ = torch.cuda.CUDAGraph()
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                with torch.cuda.graph(g_, stream=cap):
+                    body()
+            stream.wait_stream(cap)
+            torch.cuda.synchronize()
+            return g_
+
+        def with_call():
+            for _ in range(R):
+                flush.zero_()
+                fn()
+
+        def flush_only():
+            for _ in range(R):
+                flush.zero_()
+
+        gw, gf = capture(with_call), capture(flush_only)
+        tw, tf = [], []
+        for i in range(reps + 1):
+            for g_, t_ in ((gw, tw), (gf, tf)):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g_.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if i:
+                    t_.append(e0.elapsed_time(e1))
+        del gw, gf
+        return (statistics.median(tw) - statistics.median(tf)) * 1e3 / R
+
+    kern_us = {n_: diff_us(f_) for n_, f_ in comps.items()}
+    decode_device_us = diff_us(decode)
 
     # ---- the same step on the row-only cache layout (no low-dim plane) ---------
     rows_only_us = statistics.mean(timed(decode_rows_only, nb, 10)) * 1e3
@@ -460,11 +503,14 @@ def run_ours(args):
                    "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read "
                          "so no dirty lines remain), flush excluded from the timing",
                    "timing": "CUDA-graph replay of one loki_decode_attention_plane call per step, "
-                             "CUDA events on the launching stream",
+                             "CUDA events on the launching stream; decode_device_us and "
+                             "kernels_us: one graph of 8 x (L2 flush, call) minus one of 8 x "
+                             "(L2 flush), over 8 (no per-replay launch overhead)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "tokens_per_s": round(B * world * 1e6 / us_per_step_rank, 1),
         "hbm_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
         "hbm_frac_of_" + peak_kind: round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 4),
+        "decode_device_us": round(decode_device_us, 3),
         "eager_us": round(eager_us, 3),
         "rows_only_layout_eager_us": round(rows_only_us, 3),
         "dense_us": round(dense_us, 3),

@@ -81,6 +81,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
     if (warp == kScoreConsumerWarps) {
         // ---------------- producer: one lane issues every tile copy ----------------
         if (lane == 0) {
+            // the plane is read once per step: keep it from evicting the
+            // scores, which top-k reads right after this kernel
+            const uint64_t pol = l2_policy_evict_first();
             int i = 0;
             bool ok = true;
             for (int64_t r = R0; r < R1 && ok;) {
@@ -97,8 +100,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
                         break;
                     }
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(n * kRowBytes));
-                    bulk_load(ring + (size_t)st * kTile, src + (int64_t)t0 * kRowBytes,
-                              (uint32_t)(n * kRowBytes), &full[st]);
+                    bulk_load_hint(ring + (size_t)st * kTile, src + (int64_t)t0 * kRowBytes,
+                                   (uint32_t)(n * kRowBytes), &full[st], pol);
                 }
                 r += seg;
             }

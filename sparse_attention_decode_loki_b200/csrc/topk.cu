@@ -450,10 +450,11 @@ static cudaError_t launch_smem(const float* scores, int64_t rows, int S, int k, 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl) {
     const int Si = (int)S, ki = (int)k;
-    // each thread owns at most 32 consecutive keys of the row
-    if (S <= 128 * 32) return launch_smem<128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 32) return launch_smem<256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 512 * 32) return launch_smem<512>(scores, rows, Si, ki, idx, s, pdl);
+    // each thread owns at most 16 consecutive keys of the row (32 for rows
+    // longer than 16 x 512): shorter per-thread loops in a latency-bound kernel
+    if (S <= 128 * 16) return launch_smem<128>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 256 * 16) return launch_smem<256>(scores, rows, Si, ki, idx, s, pdl);
+    if (S <= 512 * 16) return launch_smem<512>(scores, rows, Si, ki, idx, s, pdl);
     if (S <= 1024 * 32) return launch_smem<1024>(scores, rows, Si, ki, idx, s, pdl);
     {
         DevInfo di;
