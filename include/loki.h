@@ -169,6 +169,25 @@ LOKI_API loki_status loki_decode_attention_plane(const void* q, const void* Kt_c
                                                  void* stream);
 
 /*
+ * The same decode step as loki_decode_attention_plane in a single kernel:
+ * one thread block per (batch, KV head) unit rotates the unit's queries,
+ * scans its key plane, keeps the scores in on-chip shared memory, selects the
+ * top k per query head and runs the sparse attention, so the scores and the
+ * selection never make a round trip through device memory. No workspace.
+ * Identical results (same selection rule, fp32 arithmetic). Limits:
+ * D = 128; H_q / H_kv in {1, 2, 4, 8}; S <= 8192; d_lo * sizeof(dt) in
+ * {16, 32, 64, 128} bytes; the unit's keys and selection must fit in shared
+ * memory. Shapes outside them return LOKI_ERR_UNSUPPORTED before any launch;
+ * other argument errors as loki_decode_attention_plane.
+ */
+LOKI_API loki_status loki_decode_attention_fused(const void* q, const void* Kt_cache,
+                                                 const void* V_cache, const void* Kt_lo, int d_lo,
+                                                 const float* P, int B, int H_q, int H_kv,
+                                                 int64_t S, int64_t S_max, int D, int d, int64_t k,
+                                                 float scale, loki_dtype dt, void* out,
+                                                 int32_t* selected_idx, void* stream);
+
+/*
  * loki_decode_attention without a workspace argument, for callers that cannot
  * allocate device memory (a plugin inside a framework that owns all device
  * allocations, a thread that must not call cudaMalloc/cudaFree because they

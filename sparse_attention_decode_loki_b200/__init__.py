@@ -22,7 +22,8 @@ from ._lib import DTYPE_BF16, DTYPE_F32, LIB_PATH, LokiError, check, lib  # noqa
 __all__ = [
     "LokiError", "LIB_PATH",
     "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
-    "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_noalloc",
+    "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_fused",
+    "loki_decode_attention_noalloc",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
     "loki_sparse_attention_workspace_size", "loki_calibrate_workspace_size",
@@ -228,6 +229,33 @@ def loki_decode_attention_plane(q, Kt_cache, V_cache, Kt_lo, P, S: int, d: int, 
     """loki_decode_attention scoring from the low-dimensional key plane Kt_lo."""
     return loki_decode_attention(q, Kt_cache, V_cache, P, S, d, k, scale, out, selected_idx,
                                  workspace, Kt_lo=Kt_lo)
+
+
+def loki_decode_attention_fused(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,
+                                Kt_lo: torch.Tensor, P: torch.Tensor, S: int, d: int, k: int,
+                                scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                selected_idx: Optional[torch.Tensor] = None
+                                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """loki_decode_attention_plane as one kernel per (batch, KV head) unit
+    (scores kept on chip; no workspace). Raises LokiError(LOKI_ERR_UNSUPPORTED)
+    for shapes outside the kernel's limits (see include/loki.h)."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q, Kt_cache, V_cache, P)
+    if out is None:
+        out = torch.empty_like(q)
+    if selected_idx is None:
+        selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    _cuda(q, out, selected_idx)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    if S > S_max:
+        raise ValueError("S must be <= S_max")
+    _check_plane(Kt_lo, Kt_cache)
+    check(lib.loki_decode_attention_fused(q.data_ptr(), Kt_cache.data_ptr(), V_cache.data_ptr(),
+                                          Kt_lo.data_ptr(), Kt_lo.shape[3], P.data_ptr(), B, H_q,
+                                          H_kv, S, S_max, D, d, k, float(scale), _dt(q),
+                                          out.data_ptr(), selected_idx.data_ptr(), _stream(dev)),
+          "loki_decode_attention_fused")
+    return out, selected_idx
 
 
 def loki_decode_attention_noalloc(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,

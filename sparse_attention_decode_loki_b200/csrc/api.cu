@@ -314,6 +314,15 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                  "workspace %zu bytes < required %zu", ws_bytes, w.total);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const loki::Dt t = to_dt(dt);
+    // Many (batch, KV head) units over a low-dim key plane: one kernel does
+    // the whole step per unit, with the scores in shared memory.
+    if (Kt_lo != nullptr && loki::decode_fused_preferred(t, B, H_q, H_kv, S, D, d_lo, k)) {
+        LOKI_CUDA(loki::launch_decode_fused(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                            S_max, d_lo, d, k, resolve_scale(scale, D), out,
+                                            selected_idx, s),
+                  name);
+        return LOKI_OK;
+    }
     float* q_rot = at<float>(ws, w.q_rot);
     float* scores = at<float>(ws, w.scores);
     int* done = at<int>(ws, w.done);
@@ -378,6 +387,36 @@ loki_status loki_decode_attention_plane(const void* q, const void* Kt_cache, con
     return decode_impl("loki_decode_attention_plane", q, Kt_cache, V_cache, Kt_lo, d_lo, P, B,
                        H_q, H_kv, S, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes,
                        stream);
+}
+
+loki_status loki_decode_attention_fused(const void* q, const void* Kt_cache, const void* V_cache,
+                                        const void* Kt_lo, int d_lo, const float* P, int B,
+                                        int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
+                                        int64_t k, float scale, loki_dtype dt, void* out,
+                                        int32_t* selected_idx, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
+    LOKI_REQUIRE(k >= 1 && k <= S, LOKI_ERR_INVALID_ARG, "k must be in [1, S] (got %lld)",
+                 (long long)k);
+    LOKI_PTR(q, 16);
+    LOKI_PTR(Kt_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(Kt_lo, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    LOKI_REQUIRE(d <= d_lo, LOKI_ERR_INVALID_ARG, "d (%d) must be <= d_lo (%d)", d, d_lo);
+    const loki::Dt t = to_dt(dt);
+    LOKI_REQUIRE(loki::decode_fused_fits(t, H_q, H_kv, S, D, d_lo, k), LOKI_ERR_UNSUPPORTED,
+                 "the fused decode kernel takes H_q / H_kv in {1, 2, 4, 8}, S <= 8192, plane "
+                 "rows of 16, 32, 64 or 128 bytes, and keys that fit in shared memory");
+    LOKI_CUDA(loki::launch_decode_fused(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S, S_max,
+                                        d_lo, d, k, resolve_scale(scale, D), out, selected_idx,
+                                        static_cast<cudaStream_t>(stream)),
+              "loki_decode_attention_fused");
+    return LOKI_OK;
 }
 
 loki_status loki_project_query(const void* q, const float* P, int B, int H_q, int H_kv, int D,

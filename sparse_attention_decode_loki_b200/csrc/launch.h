@@ -58,6 +58,21 @@ cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl);
 
+// Whether the fused one-CTA-per-unit decode kernel can run this decode over a
+// low-dim key plane: head dim 128; G in {1, 2, 4, 8}; S within the block
+// top-k; plane rows of 1, 2, 4 or 8 16-byte chunks; the unit's keys and
+// selection fit in shared memory.
+bool decode_fused_fits(Dt dt, int H_q, int H_kv, int64_t S, int D, int d_lo, int64_t k);
+// Whether loki_decode_attention_plane takes the fused kernel on its own.
+bool decode_fused_preferred(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo,
+                            int64_t k);
+// The whole decode step in one kernel: rotation, score scan over the plane,
+// top-k and sparse attention, per (batch, KV head) unit; writes out and sel.
+cudaError_t launch_decode_fused(Dt dt, const void* q, const float* P, const void* Klo,
+                                const void* Kt, const void* V, int B, int H_q, int H_kv, int64_t S,
+                                int64_t S_max, int d_lo, int d, int64_t k, float scale, void* out,
+                                int32_t* sel, cudaStream_t s);
+
 // partial slots per (batch, query head) row of the sparse attention split
 int64_t sparse_max_parts(int64_t rows, int64_t k);
 // done[B*H_q] must be zero on entry (per-row completion counters; the last

@@ -142,3 +142,22 @@ def test_python_binding_requires_cuda_tensors():
     q = torch.zeros(1, 1, 128)
     with pytest.raises(ValueError):
         loki.dense_decode_attention(q, torch.zeros(1, 1, 4, 128), torch.zeros(1, 1, 4, 128), 4)
+
+
+def test_fused_entry_point_rejects_bad_arguments(L):
+    lib = L.lib
+
+    def dec(**kw):
+        a = dict(Kt_lo=FAKE, d_lo=32, H_q=2, H_kv=2, S=100, d=32, k=10, out=FAKE)
+        a.update(kw)
+        return lib.loki_decode_attention_fused(FAKE, FAKE, FAKE, a["Kt_lo"], a["d_lo"], FAKE, 1,
+                                               a["H_q"], a["H_kv"], a["S"], 100, 128, a["d"],
+                                               a["k"], 0.0, L.DTYPE_BF16, a["out"], FAKE, None)
+    assert dec(d=33) == 1              # d > d_lo
+    assert dec(d_lo=20, d=16) == 1     # plane row not a multiple of 16 bytes
+    assert dec(Kt_lo=None) == 1
+    assert dec(k=0) == 1
+    assert dec(k=101) == 1             # k > S
+    assert dec(H_q=3) == 1             # H_q not a multiple of H_kv
+    assert dec(out=FAKE + 2) == 1      # misaligned output
+    assert L.lib.loki_last_error().decode() != ""
