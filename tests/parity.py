@@ -8,9 +8,16 @@ same bytes.
 
 Tolerances (from the spec contract of this library):
   * selected index sets are bit-exact, except for tokens whose low-dimensional
-    score lies within the tie band of the k-th score: 1e-3 relative, plus an
-    absolute floor of 1e-5 * max|s| for the case where the k-th score is
-    near zero (fp32 accumulation of d products has error ~1e-7 * sum|terms|);
+    score lies within 1e-3 relative of the k-th score. The CUDA path computes
+    q~ and the scores in fp32 (as the contract asks), and an fp32 sum cannot
+    order two tokens whose exact scores differ by less than its rounding
+    error; so a token also counts as tied when |s_j - s_k| is within the
+    forward error bound of the two fp32 scores,
+        (d + D + 2) * 2^-24 * (A_j + A_k),  A_j = sum_{i<d} |K~_ji| a_i,
+        a_i = sum_c |q_c| |P_ci|
+    (the fma-chain bound of q~ = q P over D terms, then of the d-term score).
+    Tokens that pass only through this bound are counted apart
+    (RowCheck.floor_only) and reported by the tests;
   * outputs within 2e-2 max-abs for bf16 and 1e-4 for fp32. Where the GPU set
     differs from the oracle's inside the band, the oracle attention is taken
     on the GPU's set (both sets are correct selections).
@@ -29,7 +36,7 @@ import workloads
 
 OUT_TOL = {"bf16": 2e-2, "f32": 1e-4}
 BAND_REL = 1e-3
-BAND_ABS = 1e-5
+FP32_U = 2.0 ** -24
 
 
 @dataclass
@@ -97,6 +104,16 @@ class RowCheck:
     set_equal: bool
     band_diff: int
     max_err: float
+    floor_only: int = 0
+
+
+def fp32_score_bound(q: np.ndarray, P: np.ndarray, Kt: np.ndarray, d: int) -> np.ndarray:
+    """Per-token bound on |fp32 score - exact score| for scores computed as
+    q~ = q P (D-term fp32 fma chain) then s_j = q~[:d] . K~_j[:d] (d-term chain)."""
+    D = P.shape[0]
+    a = np.abs(np.asarray(q, np.float64)) @ np.abs(np.asarray(P, np.float64))
+    A = np.abs(np.asarray(Kt, np.float64)[:, :d]) @ a[:d]
+    return (d + D + 2) * FP32_U * A
 
 
 def check_row(inp: HostInputs, b: int, h: int, gpu_idx: np.ndarray, gpu_out: np.ndarray,
@@ -108,29 +125,40 @@ def check_row(inp: HostInputs, b: int, h: int, gpu_idx: np.ndarray, gpu_out: np.
     Kt = inp.Kt[b, hk, :S].astype(np.float64)
     V = inp.V[b, hk, :S].astype(np.float64)
     P = inp.P[hk].astype(np.float64)
-    q_rot = oracle.project_query(inp.q[b, h].astype(np.float64), P)
+    q = inp.q[b, h].astype(np.float64)
+    q_rot = oracle.project_query(q, P)
     s = oracle.lowdim_scores(q_rot, Kt, d)
     I = oracle.select_topk(s, k)
     gi = np.asarray(gpu_idx, dtype=np.int64)
     assert gi.shape == (k,), gi.shape
     assert np.all(np.diff(gi) > 0), "GPU indices must be strictly ascending"
     assert gi.min() >= 0 and gi.max() < S
+    err_s = fp32_score_bound(q, P, Kt, d)
     if gpu_scores is not None:
-        atol = 1e-5 * np.abs(Kt[:, :d] * q_rot[None, :d]).sum(axis=1).max() + 1e-30
-        np.testing.assert_allclose(gpu_scores[:S], s, rtol=1e-5, atol=atol)
-    kth = s[I].min()
-    band = BAND_REL * abs(kth) + BAND_ABS * np.abs(s).max()
+        # the GPU scores obey the same forward error bound
+        dev = np.abs(np.asarray(gpu_scores[:S], np.float64) - s)
+        assert np.all(dev <= err_s + 1e-30), (
+            f"row {(b, h)}: GPU score off by {dev.max():.3e} (bound {err_s[dev.argmax()]:.3e})")
+    kpos = I[np.argmin(s[I])]
+    kth = s[kpos]
     diff = np.setxor1d(I, gi)
-    assert np.all(np.abs(s[diff] - kth) <= band), (
+    gap = np.abs(s[diff] - kth)
+    rel = BAND_REL * abs(kth)
+    floor = err_s[diff] + err_s[kpos]
+    assert np.all(gap <= rel + floor), (
         f"row {(b, h)}: {len(diff)} tokens differ outside the tie band "
-        f"(max |s-s_k| = {np.abs(s[diff] - kth).max() if len(diff) else 0:.3e}, band {band:.3e})")
+        f"(max |s-s_k| = {gap.max() if len(diff) else 0:.3e}, band {rel:.3e})")
+    floor_only = int(np.sum(gap > rel))
     ref = oracle.attend(q_rot, Kt, V, gi if len(diff) else I, scale)
     err = float(np.abs(gpu_out.astype(np.float64) - ref).max())
     assert err <= OUT_TOL[wl.dtype], f"row {(b, h)}: max |out - oracle| = {err:.3e}"
-    return RowCheck((b, h), len(diff) == 0, len(diff), err)
+    return RowCheck((b, h), len(diff) == 0, len(diff), err, floor_only)
 
 
 def summarize(checks: List[RowCheck]) -> Dict[str, float]:
-    return {"rows": len(checks), "sets_identical": sum(c.set_equal for c in checks),
-            "band_tokens": sum(c.band_diff for c in checks),
-            "max_err": max(c.max_err for c in checks)}
+    s = {"rows": len(checks), "sets_identical": sum(c.set_equal for c in checks),
+         "band_tokens": sum(c.band_diff for c in checks),
+         "floor_only_tokens": sum(c.floor_only for c in checks),
+         "max_err": max(c.max_err for c in checks)}
+    print(f"parity: {s}")
+    return s

@@ -281,3 +281,36 @@ def test_selection_prefers_high_lowdim_score_tokens_on_lowrank_keys():
     idx = oracle.select_topk(oracle.lowdim_scores(oracle.project_query(q, P), Kt, wl.d), wl.k)
     exact = oracle.select_topk(K @ q, wl.k)
     assert len(np.intersect1d(idx, exact)) >= 0.9 * wl.k
+
+
+def test_calibrate_heads_closed_form_per_head():
+    # Each head gets 8 keys +-a_i e_i, so its centred covariance is exactly
+    # diag(2 a_i^2) / (N - 1): the eigenvalues are known in closed form and
+    # the principal components are the axes sorted by variance. Head 2 is
+    # head 0 turned by 30 degrees in the (0, 1) plane, so its components are
+    # the turned axes. The per-head orders are 3-cycles, so a transposed basis
+    # or a head mix-up gives a different P.
+    a = {0: [1.0, 3.0, 2.0, 0.5], 1: [2.0, 0.5, 1.0, 3.0]}
+    D, N = 4, 8
+    th = math.radians(30.0)
+    R = np.eye(D)
+    R[0, 0], R[0, 1], R[1, 0], R[1, 1] = math.cos(th), -math.sin(th), math.sin(th), math.cos(th)
+    keys = np.zeros((N, 3, D))
+    for h in (0, 1):
+        for i in range(D):
+            keys[2 * i, h, i] = a[h][i]
+            keys[2 * i + 1, h, i] = -a[h][i]
+    keys[:, 2, :] = keys[:, 0, :] @ R.T
+    P, w = oracle.calibrate_pca_heads(keys)
+    assert P.shape == (3, D, D) and w.shape == (3, D)
+    var = {h: 2.0 * np.square(a[h]) / (N - 1) for h in (0, 1)}
+    E = np.eye(D)
+    expect_P = {
+        0: E[:, [1, 2, 0, 3]],
+        1: E[:, [3, 0, 2, 1]],
+        2: np.stack([R @ E[:, 1], E[:, 2], R @ E[:, 0], E[:, 3]], axis=1),
+    }
+    expect_w = {0: np.sort(var[0])[::-1], 1: np.sort(var[1])[::-1], 2: np.sort(var[0])[::-1]}
+    for h in range(3):
+        np.testing.assert_allclose(w[h], expect_w[h], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(P[h], expect_P[h], atol=1e-12)

@@ -62,6 +62,10 @@ def test_noalloc_matches_workspace_entry_point(cuda):
         st = L.lib.loki_decode_attention_noalloc(*args, dt, out.data_ptr(), idx.data_ptr(), stream)
         assert st == 0, (call, L.lib.loki_last_error())
         torch.cuda.synchronize()
+        # no staged kernel's bounded wait gave up during the call
+        code = ctypes.c_int(-1)
+        assert L.lib.loki_device_error(ctypes.byref(code), 1) == 0
+        assert code.value == 0, call
         idx_h = idx.cpu().numpy()
         out_h = out.float().cpu().numpy()
         assert np.array_equal(idx_h, idx_ref), call
