@@ -355,12 +355,12 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                       name);
     }
     LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
-    // attention is ordered normally after top-k (no early launch): its CTAs
-    // then start on drained SMs that take its large-L1 split
+    // attention is a programmatic dependent of top-k too: its CTAs set up
+    // their copy pipeline as SMs drain and wait for the selection
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
-                                            false),
+                                            true),
               name);
     return LOKI_OK;
 }

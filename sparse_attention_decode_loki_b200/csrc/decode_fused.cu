@@ -15,7 +15,7 @@
 //      stored as order-preserving keys in shared memory (the scores never
 //      touch HBM);
 //   2. exact radix top-k per query head over the keys in shared memory
-//      (topk_core.cuh); the selection goes to shared memory and to
+//      (topk_select.cuh); the selection goes to shared memory and to
 //      selected_idx;
 //   3. sparse attention: each warp gathers its share of one head's selected
 //      key and value rows (16-byte loads, U rows per row group in flight) with
@@ -27,7 +27,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "tma.cuh"
-#include "topk_core.cuh"
+#include "topk_select.cuh"
 
 namespace loki {
 
@@ -55,7 +55,7 @@ struct FusedLayout {
 __host__ __device__ inline FusedLayout fused_layout(int nv, int cols, int G, int S, int k) {
     const int tile = kFusedRows * nv * 16;
     int ring = kFusedStages * tile;
-    const int topk_scratch = 4096 * 4 + kTopkCandCap * 4;
+    const int topk_scratch = kTkSmemWords * 4;
     const int partials = kFusedWarps * (2 + 128) * 4;
     if (ring < topk_scratch) ring = topk_scratch;
     if (ring < partials) ring = partials;
@@ -91,8 +91,6 @@ __global__ void __launch_bounds__(kFusedThreads, MINB) k_decode_fused(
     constexpr int64_t kCacheRow = (int64_t)D * E::kBytes;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ uint64_t full[kFusedStages];
-    __shared__ int scan_buf[32];
-    __shared__ int small[5];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t unit = blockIdx.x;
@@ -228,13 +226,27 @@ __global__ void __launch_bounds__(kFusedThreads, MINB) k_decode_fused(
     }
 
     // ---- 2. top-k per query head ---------------------------------------------------
-    uint32_t* hist = reinterpret_cast<uint32_t*>(ring);
-    uint32_t* cand = hist + 4096;
+    // (the ring is free once the scan is done: it holds the selection scratch;
+    // each thread takes 8 groups of 4 keys of the head into registers)
+    const TkSmem tsm = tk_carve(reinterpret_cast<uint32_t*>(ring));
+    const TkCluster<false> one_cta;
+    constexpr int kGroups = kFusedMaxS / (4 * kFusedThreads);
+    static_assert(kGroups == 8, "fused top-k layout");
     for (int g = 0; g < G; ++g) {
-        for (int i = tid; i < 1024; i += kFusedThreads)
-            reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
-        topk_block_select<kFusedThreads>(reinterpret_cast<const uint4*>(keys + g * Spad), S, k,
-                                         sel + g * k, TopkScratch{hist, cand, scan_buf, small});
+        const uint4* kg = reinterpret_cast<const uint4*>(keys + g * Spad);
+        tk_zero<kFusedThreads>(tsm);
+        __syncthreads();
+        uint4 v[kGroups];
+#pragma unroll
+        for (int i = 0; i < kGroups; ++i) {
+            const int grp_i = warp * 32 * kGroups + 32 * i + lane;
+            v[i] = grp_i < Spad / 4 ? kg[grp_i] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (kk[e] != 0u) atomicAdd(&tsm.hist1[kk[e] >> 21], 1u);
+        }
+        tk_select<kFusedThreads, kGroups, false>(one_cta, v, 0, k, sel + g * k, tsm);
         __syncthreads();
     }
     {

@@ -43,8 +43,15 @@ __device__ __forceinline__ int64_t owner_warp(int64_t b, int64_t W, int64_t N) {
     return ((b + 1) * W - 1) / N;
 }
 
+#ifndef LOKI_SP_U
+#define LOKI_SP_U 8
+#endif
+#ifndef LOKI_SP_MINB
+#define LOKI_SP_MINB 2
+#endif
+
 template <class E>
-__global__ void __launch_bounds__(256) k_sparse_attn(
+__global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int nblk, int64_t N, int64_t W,
@@ -54,7 +61,7 @@ __global__ void __launch_bounds__(256) k_sparse_attn(
     constexpr int KV = E::kVec;
     constexpr int LPR = D / KV;     // lanes per row
     constexpr int GPW = 32 / LPR;   // row groups per warp
-    constexpr int U = 8;            // rows in flight per group
+    constexpr int U = LOKI_SP_U;    // rows in flight per group
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
     __shared__ int s_idx[8][kWarpIdx];
 

@@ -2,70 +2,91 @@
 // Insights" Figure 1 caption: keep the k tokens with the largest approximate
 // scores), as a kernel over rows of fp32 scores in global memory.
 //
-// One CTA per (batch, query head) row. Rows of up to 32768 keys
-// (k_topk_smem) load their keys into shared memory and run the block-level
-// radix select of topk_core.cuh. Longer rows (k_topk_long) keep keys in
-// shared memory, or re-read them from L2 when they do not fit, with 8-bit
-// digits and warp-aggregated atomics.
+// k_topk: each row is held in the registers of one CTA (up to 32 keys per
+// thread) or, when the row is long or there are few rows for the SMs, split
+// over the CTAs of a thread-block cluster (2, 4 or 8 CTAs) that cooperate
+// through distributed shared memory (topk_select.cuh). The first radix digit
+// is histogrammed while the scores are loaded and turned into keys. Rows too
+// long for an 8-CTA cluster (more than 262144 keys) take k_topk_long, which
+// re-reads the scores from global memory in each pass.
 #include "launch.h"
-#include "topk_core.cuh"
+#include "topk_select.cuh"
 
 namespace loki {
 
-// Rows of up to 32 * NT keys: keys in shared memory (zero-padded to a
-// multiple of 4; key 0 never comes from a score), every loop rolled and over
-// uint4 groups of 4 keys (a small kernel body that stays in the instruction
-// cache, and few instructions per key).
-template <int NT>
-__global__ void __launch_bounds__(NT) k_topk_smem(const float* __restrict__ scores, int S, int k,
-                                                  int32_t* __restrict__ out, int vec4) {
-    extern __shared__ uint4 keys4[];
-    __shared__ __align__(16) uint32_t hist[4096];
-    __shared__ uint32_t cand[kTopkCandCap];
-    __shared__ int scan_buf[32];
-    __shared__ int small[5];
-    const int tid = threadIdx.x;
-    const int S4 = (S + 3) >> 2;
-    const float* row = scores + (int64_t)blockIdx.x * S;
-#pragma unroll 1
-    for (int i = tid; i < 1024; i += NT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+constexpr int kTopkChunkTarget = 8192;  // keys per CTA the launcher aims for
+
+// One CTA (or one cluster of CTAs) per row. CTA rank r of the row's cluster
+// holds keys [r * chunk, min((r + 1) * chunk, S)); chunk is a multiple of 4
+// and at most 4 * NT * I.
+template <int NT, int I, bool kCl>
+__global__ void __launch_bounds__(NT) k_topk(const float* __restrict__ scores, int S, int k,
+                                             int chunk, int32_t* __restrict__ out, int vec4) {
+    __shared__ __align__(16) uint32_t scratch[kTkSmemWords];
+    TkCluster<kCl> cl;
+    cl.init();
+    const TkSmem sm = tk_carve(scratch);
+    tk_zero<NT>(sm);
+    __syncthreads();
     griddep_wait();  // scores come from the score kernel
     griddep_launch_dependents();
 
-    if (vec4) {  // S % 4 == 0 and scores 16-byte aligned
-        // 8 loads in flight per thread before any is used: the row arrives in
-        // one or two memory round trips instead of one per group
-        constexpr int kInFlight = 8;
-        const float4* r4 = reinterpret_cast<const float4*>(row);
-#pragma unroll 1
-        for (int j0 = tid; j0 < S4; j0 += kInFlight * NT) {
-            float4 v[kInFlight];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = blockIdx.x / cl.size;
+    const int base = cl.rank * chunk;
+    const int n = max(0, min(chunk, S - base));
+    const float* src = scores + row * S + base;
+    uint4 v[I];
 #pragma unroll
-            for (int u = 0; u < kInFlight; ++u) {
-                const int j = j0 + u * NT;
-                v[u] = j < S4 ? __ldg(r4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < kInFlight; ++u) {
-                const int j = j0 + u * NT;
-                if (j < S4)
-                    keys4[j] = make_uint4(order_key(v[u].x), order_key(v[u].y), order_key(v[u].z),
-                                          order_key(v[u].w));
-            }
-        }
-    } else {
-#pragma unroll 1
-        for (int j = tid; j < S4; j += NT) {
-            const int j4 = 4 * j;
-            keys4[j] = make_uint4(order_key(__ldg(row + j4)),
-                                  j4 + 1 < S ? order_key(__ldg(row + j4 + 1)) : 0u,
-                                  j4 + 2 < S ? order_key(__ldg(row + j4 + 2)) : 0u,
-                                  j4 + 3 < S ? order_key(__ldg(row + j4 + 3)) : 0u);
+    for (int i = 0; i < I; ++i) {
+        const int g = warp * 32 * I + 32 * i + lane;  // group of keys 4g .. 4g + 3
+        const int j = 4 * g;
+        if (vec4 && j + 3 < n) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(src) + g);
+            v[i] = make_uint4(order_key(f.x), order_key(f.y), order_key(f.z), order_key(f.w));
+        } else {
+            v[i] = make_uint4(j < n ? order_key(__ldg(src + j)) : 0u,
+                              j + 1 < n ? order_key(__ldg(src + j + 1)) : 0u,
+                              j + 2 < n ? order_key(__ldg(src + j + 2)) : 0u,
+                              j + 3 < n ? order_key(__ldg(src + j + 3)) : 0u);
         }
     }
+#pragma unroll
+    for (int i = 0; i < I; ++i) {
+        const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (kk[e] != 0u) atomicAdd(&sm.hist1[kk[e] >> 21], 1u);
+    }
+    tk_select<NT, I, kCl>(cl, v, base, k, out + row * k, sm);
+}
+
+// exclusive prefix sum over the block; `total` gets the block sum
+__device__ __forceinline__ int block_excl_scan(int v, int* buf, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = (blockDim.x + 31) >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) buf[warp] = x;
     __syncthreads();
-    topk_block_select<NT>(keys4, S, k, out + (int64_t)blockIdx.x * k,
-                          TopkScratch{hist, cand, scan_buf, small});
+    if (warp == 0) {
+        int w = lane < nw ? buf[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += y;
+        }
+        if (lane < nw) buf[lane] = w;  // inclusive warp totals
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? buf[warp - 1] : 0) + x - v;
+    *total = buf[nw - 1];
+    __syncthreads();
+    return before;
 }
 
 // Long rows: keys in shared memory (kSmem) or re-read from global memory,
@@ -149,33 +170,88 @@ __global__ void __launch_bounds__(512) k_topk_long(const float* __restrict__ sco
     }
 }
 
-template <int NT>
-static cudaError_t launch_smem(const float* scores, int64_t rows, int S, int k, int32_t* idx,
-                              cudaStream_t s, bool pdl) {
-    const size_t smem = ((size_t)S + 3) / 4 * 16;
-    if (smem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            k_topk_smem<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
+template <int NT, int I, bool kCl>
+static cudaError_t launch_rows(const float* scores, int64_t rows, int S, int k, int C, int chunk,
+                               int32_t* idx, cudaStream_t s, bool pdl) {
+    auto kern = k_topk<NT, I, kCl>;
+    cudaError_t e = prefer_carveout(reinterpret_cast<const void*>(kern),
+                                    cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const int vec4 = (S % 4 == 0) && (chunk % 4 == 0) &&
+                     (reinterpret_cast<uintptr_t>(scores) % 16 == 0);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * C));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (kCl) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)C;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
-    const int vec4 = (S % 4 == 0) && (reinterpret_cast<uintptr_t>(scores) % 16 == 0);
-    return launch_kernel(k_topk_smem<NT>, dim3((unsigned)rows), dim3(NT), smem, s, pdl, scores, S,
-                         k, idx, vec4);
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = na ? attr : nullptr;
+    cfg.numAttrs = (unsigned)na;
+    return cudaLaunchKernelEx(&cfg, kern, scores, S, k, chunk, idx, vec4);
+}
+
+template <bool kCl>
+static cudaError_t launch_shape(int nt, int gi, const float* scores, int64_t rows, int S, int k,
+                                int C, int chunk, int32_t* idx, cudaStream_t s, bool pdl) {
+#define LOKI_TK(NT_, I_) \
+    if (nt == NT_ && gi == I_) return launch_rows<NT_, I_, kCl>(scores, rows, S, k, C, chunk, idx, s, pdl);
+    LOKI_TK(128, 1) LOKI_TK(128, 2) LOKI_TK(128, 4)
+    LOKI_TK(256, 4) LOKI_TK(256, 8) LOKI_TK(512, 8) LOKI_TK(1024, 8)
+#undef LOKI_TK
+    return cudaErrorInvalidValue;
+}
+
+// Launch shape of k_topk for a [rows, S] problem: cluster size C, keys per
+// CTA (chunk), threads per CTA (nt) and groups of 4 keys per thread (gi);
+// false when S is too long for it.
+bool topk_shape(int64_t rows, int64_t S, int sm_count, int* C_out, int* chunk_out, int* nt_out,
+                int* gi_out) {
+    int C = 1;
+    auto chunk_of = [&](int c) { return (int)(((S + c - 1) / c + 3) / 4 * 4); };
+    // split a row while its CTA would hold more than the target, or while
+    // there are fewer than two CTAs per SM and the halves keep >= 1024 keys
+    while (C < kTkMaxCluster &&
+           (chunk_of(C) > kTopkChunkTarget || (rows * C < 2 * sm_count && chunk_of(2 * C) >= 1024)))
+        C *= 2;
+    const int chunk = chunk_of(C);
+    // 128 threads up to 2048 keys, then 256 threads with up to 8 groups of 4
+    // keys each, then more threads (measured: 256 x 4 beats 128 x 8 at 4096)
+    int nt = chunk > 2048 ? 256 : 128, gi = 1;
+    while (4 * nt * gi < chunk && gi < 8) gi *= 2;
+    while (4 * nt * gi < chunk && nt < 1024) nt *= 2;
+    if (4 * nt * gi < chunk) return false;
+    *C_out = C;
+    *chunk_out = chunk;
+    *nt_out = nt;
+    *gi_out = gi;
+    return true;
 }
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl) {
     const int Si = (int)S, ki = (int)k;
-    // each thread owns at most 16 consecutive keys of the row (32 for rows
-    // longer than 16 x 512): shorter per-thread loops in a latency-bound kernel
-    if (S <= 128 * 16) return launch_smem<128>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 256 * 16) return launch_smem<256>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 512 * 16) return launch_smem<512>(scores, rows, Si, ki, idx, s, pdl);
-    if (S <= 1024 * 32) return launch_smem<1024>(scores, rows, Si, ki, idx, s, pdl);
+    DevInfo di;
+    cudaError_t e = dev_info(&di);
+    if (e != cudaSuccess) return e;
+    int C, chunk, nt, gi;
+    if (topk_shape(rows, S, di.sm_count, &C, &chunk, &nt, &gi)) {
+        if (C == 1) return launch_shape<false>(nt, gi, scores, rows, Si, ki, 1, chunk, idx, s, pdl);
+        return launch_shape<true>(nt, gi, scores, rows, Si, ki, C, chunk, idx, s, pdl);
+    }
     {
-        DevInfo di;
-        cudaError_t e = dev_info(&di);
-        if (e != cudaSuccess) return e;
         const size_t need = (size_t)S * 4;
         if (need + 4096 <= (size_t)di.smem_optin) {
             e = cudaFuncSetAttribute(k_topk_long<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
