@@ -39,7 +39,7 @@ if ROOT not in sys.path:
 METRIC = "Loki decode-attn µs/layer-step, HBM GB/s (% roofline), speedup vs dense"
 UNIT = "us/layer-step"
 FALLBACK_HBM_GBS = 6650.0
-LAUNCHES_PER_DECODE = 4  # projection, score scan, top-k, sparse attention with its row merge
+LAUNCHES_PER_DECODE = 4  # score scan, projection, top-k, sparse attention with its row merge
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB of L2
 
 
@@ -108,7 +108,8 @@ def host_cores():
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML every 5 ms."""
+    """Samples SM clock and throttle reasons through NVML every 2 ms (from the
+    start of warm-up to the end of the timed region)."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
@@ -148,7 +149,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
@@ -226,24 +227,36 @@ def blas_threads():
         return 1
 
 
-def cpu_oracle_time(wl, seconds: float, rows_per_step: int = 0):
-    """Time oracle.loki_decode_row over sampled rows; returns (us per layer-step, info)."""
+def cpu_oracle_time(wl, seconds: float, threads: int = 0):
+    """Time oracle.loki_decode_row over sampled rows; returns (us per layer-step, info).
+    threads > 0 limits the BLAS threads for the measurement."""
+    import contextlib
+
     import oracle
     sample = oracle_sample_rows(wl, 8)
+    limit = contextlib.nullcontext()
+    if threads:
+        try:
+            from threadpoolctl import threadpool_limits
+            limit = threadpool_limits(limits=threads, user_api="blas")
+        except Exception:
+            pass
     per_row = []
-    t_end = time.perf_counter() + seconds
-    i = 0
-    while (time.perf_counter() < t_end or len(per_row) < 4) and len(per_row) < 100000:
-        q, Kt, V, P = sample[i % len(sample)]
-        t0 = time.perf_counter()
-        oracle.loki_decode_row(q, Kt, V, P, wl.d, wl.k, wl.scale)
-        per_row.append(time.perf_counter() - t0)
-        i += 1
+    with limit:
+        used = blas_threads()
+        t_end = time.perf_counter() + seconds
+        i = 0
+        while (time.perf_counter() < t_end or len(per_row) < 4) and len(per_row) < 100000:
+            q, Kt, V, P = sample[i % len(sample)]
+            t0 = time.perf_counter()
+            oracle.loki_decode_row(q, Kt, V, P, wl.d, wl.k, wl.scale)
+            per_row.append(time.perf_counter() - t0)
+            i += 1
     mean_row = sum(per_row) / len(per_row)
     rows = wl.B * wl.H_q
     return mean_row * rows * 1e6, {
         "rows_timed": len(per_row), "distinct_rows": len(sample),
-        "cores": blas_threads(), "host_cores": host_cores()}
+        "cores": used, "host_cores": host_cores()}
 
 
 # ---------------------------------------------------------------------------
@@ -252,7 +265,6 @@ def cpu_oracle_time(wl, seconds: float, rows_per_step: int = 0):
 
 def build_gpu_inputs(wl, dev, rank):
     """Seeded inputs on the device; P and the rotated cache come from the library."""
-    import numpy as np
     import torch
 
     import sparse_attention_decode_loki_b200 as loki
@@ -280,6 +292,58 @@ def build_gpu_inputs(wl, dev, rank):
             "V_new": V_new, "q_host": g["q"]}
 
 
+L2_BYTES = 126 << 20
+
+
+def layer_count(hot_bytes: int, layer_bytes: int, free_bytes: int, max_layers: int = 64) -> int:
+    """Distinct layer caches to cycle through so that consecutive steps never
+    find their inputs in L2: enough layers that the others' hot bytes between
+    two visits of a layer are at least twice the L2 size, within half the
+    free device memory. 1 means the steps must flush L2 instead."""
+    if hot_bytes <= 0:
+        return 1
+    need = 1 + -(-2 * L2_BYTES // hot_bytes)
+    if hot_bytes >= L2_BYTES:
+        need = max(2, min(need, 4))
+    fit = int(0.5 * free_bytes // max(layer_bytes, 1))
+    n = min(need, fit, max_layers)
+    return n if n >= need else 1
+
+
+NOMINAL_HBM_BYTES = 180e9
+
+
+def workload_config(wl, n_layers: int, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D, "S": wl.S,
+            "d": wl.d, "k": wl.k, "cache_dtype": wl.dtype,
+            "cache_layout": "rotated K rows + contiguous d-column key plane",
+            "layers": n_layers,
+            "l2": ("inputs larger than L2: consecutive steps cycle through "
+                   f"{n_layers} distinct layer caches ({wl.loki_bytes() / 1e6:.1f} MB of "
+                   "hot bytes each), no flush" if n_layers > 1 else
+                   "flushed before every step (256 MiB write, then a 256 MiB read so "
+                   "no dirty lines remain), flush excluded"),
+            "timing": "K consecutive layer-steps (one loki_decode_attention_plane call "
+                      "each) captured in CUDA graphs and replayed back to back, CUDA "
+                      "events on the launching stream around all K",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def layer_bytes_of(wl) -> int:
+    return wl.elem_bytes * wl.B * wl.H_kv * wl.S * (2 * wl.D + wl.d)
+
+
+def actual_bytes_per_step(workload: str):
+    """DRAM bytes of one decode step as ncu counted them (sum over the step's
+    kernels), from the committed profile summaries whose sources still match."""
+    names = ["score_plane", "topk", "sparse_attn", "project_query"]
+    vals = [traffic_from_profiles(n, workload) for n in names]
+    if any(v is None for v in vals):
+        return None
+    return sum(vals)
+
+
 def run_ours(args):
     import torch
 
@@ -298,124 +362,74 @@ def run_ours(args):
     q, Kt, V, P, Kt_lo = inp["q"], inp["Kt"], inp["V"], inp["P"], inp["Kt_lo"]
     B, H_q, H_kv, S, D, d, k = wl.B, wl.H_q, wl.H_kv, wl.S, wl.D, wl.d, wl.k
     e = wl.elem_bytes
-    out = torch.empty_like(q)
-    idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cap = torch.cuda.Stream(dev)
+
+    # ---- layers: distinct copies of the cache, so consecutive steps never hit L2 --
+    free, _ = torch.cuda.mem_get_info(dev)
+    n_layers = layer_count(wl.loki_bytes(), layer_bytes_of(wl), free)
+    layers = [(Kt, V, Kt_lo)] + [(Kt.clone(), V.clone(), Kt_lo.clone())
+                                 for _ in range(n_layers - 1)]
+    outs = [torch.empty_like(q) for _ in range(n_layers)]
+    idxs = [torch.empty((B, H_q, k), dtype=torch.int32, device=dev) for _ in range(n_layers)]
     ws = torch.empty(loki.loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k),
                      dtype=torch.uint8, device=dev)
+    out, idx = outs[0], idxs[0]
+
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
-    class _Flush:
-        """Evict L2 before a timed step: write 256 MiB (the write-flush), then read
-        another 256 MiB so the dirty lines are written back here, outside the timed
-        region, and the step starts with a cold, clean L2."""
+    def flush():
+        """Evict L2: write 256 MiB, then read another 256 MiB so the dirty lines
+        are written back here and the next call starts with a cold, clean L2."""
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=flush_sink)
 
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            torch.sum(flush_r, dim=0, out=flush_sink)
+    def decode_layer(j):
+        Ktj, Vj, Kloj = layers[j]
+        loki.loki_decode_attention(q, Ktj, Vj, P, S, d, k, wl.scale, out=outs[j],
+                                   selected_idx=idxs[j], workspace=ws, Kt_lo=Kloj)
 
-    flush = _Flush()
-
-    def decode():
-        loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
-                                   workspace=ws, Kt_lo=Kt_lo)
-
-    def decode_rows_only():
-        loki.loki_decode_attention(q, Kt, V, P, S, d, k, wl.scale, out=out, selected_idx=idx,
-                                   workspace=ws)
-
-    def timed(fn, n, warm):
-        for _ in range(warm):
-            flush.zero_()
-            fn()
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for i in range(n):
-            flush.zero_()
-            starts[i].record(stream)
-            fn()
-            ends[i].record(stream)
+    def capture(body):
+        g_ = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g_, stream=cap):
+                body()
+        stream.wait_stream(cap)
         torch.cuda.synchronize()
-        return [s.elapsed_time(t) for s, t in zip(starts, ends)]
+        return g_
 
-    # One decode call is captured once into a CUDA graph: the replay launches
-    # exactly the kernels the call launches (same C-ABI call, same arguments),
-    # without the Python/ctypes issue time between them.
-    decode()
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream(dev)
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap):
-            decode()
-    stream.wait_stream(cap)
-    torch.cuda.synchronize()
+    def step_graphs(fn_layer, steps):
+        """Graphs that together run exactly `steps` consecutive layer-steps
+        (layers cycling; an L2 flush before each step when there is one layer)."""
+        def body(n):
+            def run():
+                for i in range(n):
+                    if n_layers == 1:
+                        flush()
+                    fn_layer(i % n_layers)
+            return run
+        per = max(n_layers, 1)
+        plan = [per] * (steps // per) + ([steps % per] if steps % per else [])
+        graphs = {n_: capture(body(n_)) for n_ in set(plan)}
+        return plan, graphs
 
-    # ---- the timed region: exactly K decode steps --------------------------------
-    for _ in range(args.warmup):
-        flush.zero_()
-        graph.replay()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        step_ms = timed(graph.replay, args.steps, 0)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    total_ms = max_over_ranks(sum(step_ms), world, dev)
-    us_per_step_rank = total_ms * 1e3 / args.steps
-    value = whole_job_us_per_step(total_ms, args.steps, world)
-    nb = max(50, min(args.steps, 400))
-    eager_us = statistics.mean(timed(decode, nb, 10)) * 1e3
-
-    # ---- per-kernel times: each step entry point alone, after an L2 flush -------
-    q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
-    scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
-    sp_ws = torch.empty(loki.loki_sparse_attention_workspace_size(B, H_q, k, D), dtype=torch.uint8,
-                        device=dev)
-    loki.loki_project_query(q, P, q_rot)
-    loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores)
-    loki.loki_topk(scores, k, idx)
-    comps = {
-        "project_query": lambda: loki.loki_project_query(q, P, q_rot),
-        "score_lowdim": lambda: loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores),
-        "topk": lambda: loki.loki_topk(scores, k, idx),
-        "sparse_attention+combine": lambda: loki.loki_sparse_attention(q_rot, Kt, V, idx, S,
-                                                                       wl.scale, out, sp_ws),
-    }
-    # (the decode call fuses the rotation into the score kernel and the merge
-    # into the attention kernel; the step entry points time them separately).
-    # Device time of one call with a cold L2, without the per-replay launch
-    # overhead of a graph: one graph holds R x (L2 flush, call), another R x
-    # (L2 flush); the difference of their CUDA-event times over R is the
-    # call's time, its launch gaps inside a graph included.
     def diff_us(fn, R=8, reps=5):
+        """Device time of one call with a cold L2, without per-replay launch
+        overhead: a graph of R x (L2 flush, call) minus one of R x (L2 flush)."""
         fn()
         torch.cuda.synchronize()
 
-        def capture(body):
-            g_ = torch.cuda.CUDAGraph()
-            cap.wait_stream(stream)
-            with torch.cuda.stream(cap):
-                with torch.cuda.graph(g_, stream=cap):
-                    body()
-            stream.wait_stream(cap)
-            torch.cuda.synchronize()
-            return g_
-
         def with_call():
             for _ in range(R):
-                flush.zero_()
+                flush()
                 fn()
 
         def flush_only():
             for _ in range(R):
-                flush.zero_()
+                flush()
 
         gw, gf = capture(with_call), capture(flush_only)
         tw, tf = [], []
@@ -432,46 +446,163 @@ def run_ours(args):
         del gw, gf
         return (statistics.median(tw) - statistics.median(tf)) * 1e3 / R
 
+    # ---- the timed region: exactly K layer-steps ------------------------------------
+    decode_layer(0)
+    torch.cuda.synchronize()
+    plan, graphs = step_graphs(decode_layer, args.steps)
+    wplan, wgraphs = step_graphs(decode_layer, max(args.warmup, 1))
+    with ClockSampler(local) as clk:
+        for n_ in wplan:
+            wgraphs[n_].replay()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for n_ in plan:
+            graphs[n_].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+    timed_ms = e0.elapsed_time(e1)
+    del graphs, wgraphs
+    if n_layers == 1:
+        # one layer: every step began with an L2 flush; time the same number of
+        # flushes alone and take them out (they are not part of the step)
+        fplan, fgraphs = step_graphs(lambda j: None, args.steps)
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1_ = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for n_ in fplan:
+            fgraphs[n_].replay()
+        g1_.record(stream)
+        torch.cuda.synchronize()
+        timed_ms -= g0.elapsed_time(g1_)
+        del fgraphs
+    total_ms = max_over_ranks(timed_ms, world, dev)
+    us_per_step_rank = total_ms * 1e3 / args.steps
+    value = whole_job_us_per_step(total_ms, args.steps, world)
+
+    # ---- the same step, one layer, as a single graph replay after an L2 flush -------
+    g1 = capture(lambda: decode_layer(0))
+    single = []
+    for i in range(min(200, max(20, args.steps)) + 3):
+        flush()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        g1.replay()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            single.append(a0.elapsed_time(a1) * 1e3)
+    del g1
+    decode_device_us = diff_us(lambda: decode_layer(0))
+
+    # ---- per-kernel device times: each step entry point alone, after an L2 flush ----
+    q_rot = torch.empty((B, H_q, D), dtype=torch.float32, device=dev)
+    scores = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
+    sp_ws = torch.empty(loki.loki_sparse_attention_workspace_size(B, H_q, k, D), dtype=torch.uint8,
+                        device=dev)
+    loki.loki_project_query(q, P, q_rot)
+    loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores)
+    loki.loki_topk(scores, k, idx)
+    comps = {
+        "project_query": lambda: loki.loki_project_query(q, P, q_rot),
+        "score_lowdim": lambda: loki.loki_score_lowdim(q_rot, Kt_lo, S, d, scores),
+        "topk": lambda: loki.loki_topk(scores, k, idx),
+        "sparse_attention+combine": lambda: loki.loki_sparse_attention(q_rot, Kt, V, idx, S,
+                                                                       wl.scale, out, sp_ws),
+    }
     kern_us = {n_: diff_us(f_) for n_, f_ in comps.items()}
-    decode_device_us = diff_us(decode)
 
-    # ---- the same step on the row-only cache layout (no low-dim plane) ---------
-    rows_only_us = statistics.mean(timed(decode_rows_only, nb, 10)) * 1e3
-    del graph
+    # ---- the single-kernel variant, where the shape fits it -----------------------
+    fused_us = None
+    try:
+        loki.loki_decode_attention_fused(q, Kt, V, Kt_lo, P, S, d, k, wl.scale, out=out,
+                                         selected_idx=idx)
+        torch.cuda.synchronize()
+        fused_us = diff_us(lambda: loki.loki_decode_attention_fused(
+            q, Kt, V, Kt_lo, P, S, d, k, wl.scale, out=out, selected_idx=idx))
+    except loki.LokiError:
+        pass
 
-    # ---- dense baseline on the same cache (q~ rounded to the cache dtype) ------
+    # ---- dense baseline on the same caches, timed like the headline ---------------
     q_rot_dt = loki.loki_project_query(q, P).to(q.dtype)
     dws = torch.empty(loki.dense_decode_workspace_size(B, H_q, H_kv, S, D), dtype=torch.uint8,
                       device=dev)
     dout = torch.empty_like(q)
-    dense_ms = timed(lambda: loki.dense_decode_attention(q_rot_dt, Kt, V, S, wl.scale, dout, dws),
-                     nb, 10)
-    dense_us = statistics.mean(dense_ms) * 1e3
 
-    # ---- append of one new token per (sequence, KV head) -------------------------
+    def dense_layer(j):
+        loki.dense_decode_attention(q_rot_dt, layers[j][0], layers[j][1], S, wl.scale, dout, dws)
+
+    dense_layer(0)
+    dsteps = max(n_layers, min(args.steps, 200))
+    dplan, dgraphs = step_graphs(dense_layer, dsteps)
+    for n_ in dplan[:1]:
+        dgraphs[n_].replay()
+    torch.cuda.synchronize()
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for n_ in dplan:
+        dgraphs[n_].replay()
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_us = d0.elapsed_time(d1) * 1e3 / dsteps
+    del dgraphs
+    dense_device_us = diff_us(lambda: dense_layer(0))
+
+    # ---- append of one new token per (sequence, KV head), device time ---------------
     Kt_app = torch.empty((B, H_kv, 8, D), dtype=q.dtype, device=dev)
     V_app = torch.empty_like(Kt_app)
-    app_ms = timed(lambda: loki.loki_append_keys(inp["K_new"], inp["V_new"], P, Kt_app, V_app, 0),
-                   nb, 10)
-    append_us = statistics.mean(app_ms) * 1e3
+    append_us = diff_us(lambda: loki.loki_append_keys(inp["K_new"], inp["V_new"], P, Kt_app,
+                                                      V_app, 0))
 
     # ---- end to end through the public API with host buffers ---------------------
     q_pin = torch.from_numpy(inp["q_host"]).to(q.dtype).pin_memory()
     out_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     idx_pin = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
 
-    def e2e_step():
+    def e2e_step(j):
+        if n_layers == 1:
+            flush()
         q.copy_(q_pin, non_blocking=True)
-        decode()
-        out_pin.copy_(out, non_blocking=True)
-        idx_pin.copy_(idx, non_blocking=True)
+        decode_layer(j)
+        out_pin.copy_(outs[j], non_blocking=True)
+        idx_pin.copy_(idxs[j], non_blocking=True)
 
-    e2e_ms = timed(e2e_step, max(50, min(args.steps, 1000)), 5)
-    e2e_us = max_over_ranks(statistics.mean(e2e_ms) * 1e3, world, dev)
+    n_e2e = max(20, min(args.steps, 1000))
+    for j in range(3):
+        e2e_step(j % n_layers)
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(n_e2e):
+        e2e_step(i % n_layers)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / n_e2e
+    if n_layers == 1:  # the flushes are not part of the step
+        fl = capture(lambda: flush())
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(50):
+            fl.replay()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms -= c0.elapsed_time(c1) / 50
+        del fl
+    e2e_us = max_over_ranks(e2e_ms * 1e3, world, dev)
     h2d = q_pin.numel() * q_pin.element_size()
     d2h = out_pin.numel() * out_pin.element_size() + idx_pin.numel() * idx_pin.element_size()
 
-    # ---- roofline of the dominant kernel ------------------------------------------
+    # ---- roofline of the dominant kernel and of the whole step -------------------
     peak, peak_kind = load_peaks()
     alg = {
         "score_lowdim": e * B * H_kv * S * d,
@@ -480,9 +611,9 @@ def run_ours(args):
     dom = max(alg, key=lambda n: kern_us[n])
     achieved = alg[dom] / (kern_us[dom] * 1e-6) / 1e9
     step_bytes = wl.loki_bytes()
-    step_us = us_per_step_rank
     prof_name = {"score_lowdim": "score_plane", "sparse_attention+combine": "sparse_attn"}[dom]
     traffic = traffic_from_profiles(prof_name, wl.name)
+    actual = actual_bytes_per_step(wl.name)
 
     res = {
         "metric": METRIC,
@@ -497,25 +628,24 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16" if wl.dtype == "bf16" else "f32",
         "data": "synthetic (seeded low-rank keys, N(0,1) values; PCA and cache built by the library)",
-        "config": {"workload": wl.name, "B": B, "H_q": H_q, "H_kv": H_kv, "D": D, "S": S,
-                   "d": d, "k": k, "cache_dtype": wl.dtype,
-                   "cache_layout": "rotated K rows + contiguous d-column key plane",
-                   "l2": "flushed before every timed step (256 MiB write, then a 256 MiB read "
-                         "so no dirty lines remain), flush excluded from the timing",
-                   "timing": "CUDA-graph replay of one loki_decode_attention_plane call per step, "
-                             "CUDA events on the launching stream; decode_device_us and "
-                             "kernels_us: one graph of 8 x (L2 flush, call) minus one of 8 x "
-                             "(L2 flush), over 8 (no per-replay launch overhead)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": workload_config(wl, n_layers, world),
+        "timing_detail": "single_layer_*: one call per graph replay after an L2 flush; "
+                         "*_device_us and kernels_us: graph of 8 x (L2 flush, call) minus "
+                         "graph of 8 x (L2 flush), over 8",
         "tokens_per_s": round(B * world * 1e6 / us_per_step_rank, 1),
-        "hbm_gbs": round(step_bytes / (step_us * 1e-6) / 1e9, 1),
-        "hbm_frac_of_" + peak_kind: round(step_bytes / (step_us * 1e-6) / 1e9 / peak, 4),
+        "hbm_gbs": round(step_bytes / (us_per_step_rank * 1e-6) / 1e9, 1),
+        "hbm_frac_of_" + peak_kind: round(step_bytes / (us_per_step_rank * 1e-6) / 1e9 / peak, 4),
+        "hbm_frac_actual_of_" + peak_kind: (None if actual is None else round(
+            actual / (us_per_step_rank * 1e-6) / 1e9 / peak, 4)),
+        "actual_bytes_per_step": actual,
+        "ideal_bytes_per_step": step_bytes,
+        "single_layer_graph_us": round(statistics.mean(single), 3),
         "decode_device_us": round(decode_device_us, 3),
-        "eager_us": round(eager_us, 3),
-        "rows_only_layout_eager_us": round(rows_only_us, 3),
+        "fused_kernel_device_us": None if fused_us is None else round(fused_us, 3),
         "dense_us": round(dense_us, 3),
-        "speedup_vs_dense": round(dense_us / step_us, 3),
-        "append_us": round(append_us, 3),
+        "dense_device_us": round(dense_device_us, 3),
+        "speedup_vs_dense": round(dense_us / us_per_step_rank, 3),
+        "append_device_us": round(append_us, 3),
         "kernels_us": {n_: round(v_, 3) for n_, v_ in kern_us.items()},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -528,12 +658,14 @@ def run_ours(args):
     }
     if rank == 0 and not args.no_cpu_baseline:
         cpu_us, info = cpu_oracle_time(wl, args.cpu_seconds)
+        cpu1_us, info1 = cpu_oracle_time(wl, min(4.0, args.cpu_seconds), threads=1)
         res["cpu_baseline"] = {"value": round(cpu_us, 1), "unit": UNIT, "cores": info["cores"],
                                "kind": "oracle",
-                               "sample": f"{info['rows_timed']} timed (batch, head) rows drawn "
-                                         f"from {info['distinct_rows']} seeded rows of "
-                                         f"{wl.name}, scaled by B*H_q = {B * H_q}",
-                               "host_cores": info["host_cores"]}
+                               "sample": f"extrapolated: {info['rows_timed']} timed (batch, head) "
+                                         f"rows drawn from {info['distinct_rows']} seeded rows "
+                                         f"of {wl.name}, mean row time x B*H_q = {B * H_q}",
+                               "host_cores": info["host_cores"],
+                               "one_thread_value": round(cpu1_us, 1)}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -542,14 +674,28 @@ def run_ours(args):
 
 
 def run_reference(args):
+    """The fp64 oracle on the host cores as the reference arm: each step runs
+    B * H_q row decodes (cycling through seeded sampled rows of the workload)
+    when the whole run fits in about two minutes, else a bounded sample of
+    rows per step, scaled to B * H_q and labelled as extrapolated."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     import workloads
     wl = workloads.get(args.workload)
-    rows_per_step = 4
     import oracle
     sample = oracle_sample_rows(wl, 8)
+    rows_full = wl.B * wl.H_q
+    t0 = time.perf_counter()
+    for q, Kt, V, P in sample:
+        oracle.loki_decode_row(q, Kt, V, P, wl.d, wl.k, wl.scale)
+    t_row = (time.perf_counter() - t0) / len(sample)
+    budget_s = 120.0
+    steps_all = args.steps + args.warmup
+    if steps_all * rows_full * t_row <= budget_s:
+        rows_per_step = rows_full
+    else:
+        rows_per_step = max(1, int(budget_s / (steps_all * t_row)))
 
     def step(i):
         for j in range(rows_per_step):
@@ -562,17 +708,21 @@ def run_reference(args):
     for i in range(args.steps):
         step(i)
     dt = time.perf_counter() - t0
-    per_row = dt / (args.steps * rows_per_step)
-    us = per_row * wl.B * wl.H_q * 1e6
-    sample_txt = (f"{rows_per_step} (batch, head) rows per step from 8 seeded rows of {wl.name}, "
-                  f"scaled by B*H_q = {wl.B * wl.H_q}")
+    us = dt / args.steps * (rows_full / rows_per_step) * 1e6
+    if rows_per_step == rows_full:
+        sample_txt = (f"full steps: {rows_full} (batch, head) row decodes per step, cycling "
+                      f"through {len(sample)} seeded rows of {wl.name}")
+    else:
+        sample_txt = (f"extrapolated: {rows_per_step} (batch, head) rows per step from "
+                      f"{len(sample)} seeded rows of {wl.name}, scaled by B*H_q / "
+                      f"{rows_per_step} = {rows_full / rows_per_step:.1f}")
+    n_layers = layer_count(wl.loki_bytes(), layer_bytes_of(wl), int(NOMINAL_HBM_BYTES))
     res = {
         "metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded low-rank keys)", "impl": "reference",
-        "config": {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D,
-                   "S": wl.S, "d": wl.d, "k": wl.k, "cache_dtype": wl.dtype},
+        "config": workload_config(wl, n_layers, world),
         "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": blas_threads(),
                          "kind": "oracle", "sample": sample_txt},
         "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -610,8 +760,28 @@ def run_ncu_case(args):
     torch.cuda.synchronize()
 
 
+def relaunch_ranks(n: int) -> int:
+    """Run this command as n ranks (one process per GPU) under torch.distributed.run."""
+    import subprocess
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks and let them print
+        sys.exit(relaunch_ranks(args.gpus))
+    _, world, _ = dist_env()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; using {world} ranks",
+              file=sys.stderr)
     if args.ncu_case:
         run_ncu_case(args)
         return

@@ -43,6 +43,68 @@ __device__ __forceinline__ int64_t owner_warp(int64_t b, int64_t W, int64_t N) {
     return ((b + 1) * W - 1) / N;
 }
 
+// Issue the key and value loads of one batch: U rows per row group, rows
+// jb + u * GPW + grp of the staged index list (indices past n, or -1 for an
+// index outside [0, S), load nothing and give zeros).
+template <int U, int GPW>
+__device__ __forceinline__ void sp_load(const int* widx, int n, int jb, int grp, const char* Kb,
+                                        const char* Vb, int64_t row_bytes, int (&t)[U],
+                                        uint4 (&kv)[U], uint4 (&vv)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int jj = jb + u * GPW + grp;
+        const int tok = jj < n ? widx[jj] : -1;
+        t[u] = tok;
+        if (tok >= 0) {
+            kv[u] = ld_stream(Kb + (int64_t)tok * row_bytes);
+            vv[u] = ld_stream(Vb + (int64_t)tok * row_bytes);
+        } else {
+            kv[u] = make_uint4(0u, 0u, 0u, 0u);
+            vv[u] = kv[u];
+        }
+    }
+}
+
+// Fold one loaded batch into the row group's running softmax state (m, l,
+// acc) in base 2: full-D scores, then the value rows weighted by 2^(s - m).
+template <class E, int U, int LPR>
+__device__ __forceinline__ void sp_consume(const float (&qv)[E::kVec], const int (&t)[U],
+                                           const uint4 (&kv)[U], const uint4 (&vv)[U], float& m,
+                                           float& l, float (&acc)[E::kVec]) {
+    constexpr int KV = E::kVec;
+    float sc[U];
+    float mx = m;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float f[KV];
+        E::unpack(kv[u], f);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
+        a = group_sum<LPR>(a);
+        sc[u] = t[u] >= 0 ? a : -INFINITY;
+        mx = fmaxf(mx, sc[u]);
+    }
+    if (mx == -INFINITY) return;  // nothing in this batch for this row group
+    const float alpha = exp2f(m - mx);
+    l *= alpha;
+#pragma unroll
+    for (int e = 0; e < KV; ++e) acc[e] *= alpha;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const float p = exp2f(sc[u] - mx);
+        l += p;
+        float f[KV];
+        E::unpack(vv[u], f);
+#pragma unroll
+        for (int e = 0; e < KV; ++e) acc[e] = fmaf(p, f[e], acc[e]);
+    }
+    m = mx;
+}
+
+#ifndef LOKI_SP_PIPE
+#define LOKI_SP_PIPE 0
+#endif
 #ifndef LOKI_SP_U
 #define LOKI_SP_U 8
 #endif
@@ -107,51 +169,27 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
                 widx[t] = ((unsigned)tok < (unsigned)S) ? tok : -1;
             }
             __syncwarp();
+#if LOKI_SP_PIPE
+            // two batches in registers: the next batch's loads are in flight
+            // while the current one is folded in
+            constexpr int STEP = GPW * U;
+            int tA[U], tB[U];
+            uint4 kA[U], vA[U], kB[U], vB[U];
+            sp_load<U, GPW>(widx, n, 0, grp, Kb, Vb, kRowBytes, tA, kA, vA);
+            for (int jb = 0; jb < n; jb += 2 * STEP) {
+                sp_load<U, GPW>(widx, n, jb + STEP, grp, Kb, Vb, kRowBytes, tB, kB, vB);
+                sp_consume<E, U, LPR>(qv, tA, kA, vA, m, l, acc);
+                sp_load<U, GPW>(widx, n, jb + 2 * STEP, grp, Kb, Vb, kRowBytes, tA, kA, vA);
+                sp_consume<E, U, LPR>(qv, tB, kB, vB, m, l, acc);
+            }
+#else
             for (int jb = 0; jb < n; jb += GPW * U) {
                 int t[U];
                 uint4 kv[U], vv[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int jj = jb + u * GPW + grp;
-                    const int tok = jj < n ? widx[jj] : -1;
-                    t[u] = tok;
-                    if (tok >= 0) {
-                        kv[u] = ld_stream(Kb + (int64_t)tok * kRowBytes);
-                        vv[u] = ld_stream(Vb + (int64_t)tok * kRowBytes);
-                    } else {
-                        kv[u] = make_uint4(0u, 0u, 0u, 0u);
-                        vv[u] = kv[u];
-                    }
-                }
-                float sc[U];
-                float mx = m;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    float f[KV];
-                    E::unpack(kv[u], f);
-                    float a = 0.f;
-#pragma unroll
-                    for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
-                    a = group_sum<LPR>(a);
-                    sc[u] = t[u] >= 0 ? a : -INFINITY;
-                    mx = fmaxf(mx, sc[u]);
-                }
-                if (mx == -INFINITY) continue;
-                const float alpha = exp2f(m - mx);
-                l *= alpha;
-#pragma unroll
-                for (int e = 0; e < KV; ++e) acc[e] *= alpha;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const float p = exp2f(sc[u] - mx);
-                    l += p;
-                    float f[KV];
-                    E::unpack(vv[u], f);
-#pragma unroll
-                    for (int e = 0; e < KV; ++e) acc[e] = fmaf(p, f[e], acc[e]);
-                }
-                m = mx;
+                sp_load<U, GPW>(widx, n, jb, grp, Kb, Vb, kRowBytes, t, kv, vv);
+                sp_consume<E, U, LPR>(qv, t, kv, vv, m, l, acc);
             }
+#endif
         }
         // merge the warp's row groups (lane l and lane l + LPR hold the same columns)
 #pragma unroll
@@ -198,26 +236,40 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
         prev = __shfl_sync(0xffffffffu, prev, 0);
         if (prev == nparts - 1) {
             __threadfence();
+            // lanes share the parts: (m, l) of part p go to lane p % 32, and
+            // lane l merges columns [4 l, 4 l + 4) over all parts with eight
+            // loads in flight at a time
             const float2* ml = part_ml + r + wf;
             const float* pacc = part_acc + (r + wf) * D;
             float M = -INFINITY;
-            for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(&ml[p].x));
-            float Lsum = 0.f, A[D / 32];
+            for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(&ml[p].x));
 #pragma unroll
-            for (int e = 0; e < D / 32; ++e) A[e] = 0.f;
+            for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            float Lsum = 0.f;
+            float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
             if (M != -INFINITY) {
-                for (int p = 0; p < nparts; ++p) {
+                for (int p = lane; p < nparts; p += 32) {
                     const float2 mlp = __ldcg(&ml[p]);
-                    const float sc = exp2f(mlp.x - M);
-                    Lsum += mlp.y * sc;
-                    const float* pa = pacc + (int64_t)p * D;
-#pragma unroll
-                    for (int e = 0; e < D / 32; ++e) A[e] += __ldcg(pa + e * 32 + lane) * sc;
+                    Lsum += mlp.y * exp2f(mlp.x - M);
+                }
+#pragma unroll 8
+                for (int p = 0; p < nparts; ++p) {
+                    const float sc = exp2f(__ldcg(&ml[p].x) - M);
+                    const float4 a = __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane);
+                    A.x = fmaf(a.x, sc, A.x);
+                    A.y = fmaf(a.y, sc, A.y);
+                    A.z = fmaf(a.z, sc, A.z);
+                    A.w = fmaf(a.w, sc, A.w);
                 }
             }
-            const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
 #pragma unroll
-            for (int e = 0; e < D / 32; ++e) out[r * D + e * 32 + lane] = E::from_float(A[e] * inv);
+            for (int off = 16; off >= 1; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+            const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+            typename E::T* o = out + r * D + 4 * lane;
+            o[0] = E::from_float(A.x * inv);
+            o[1] = E::from_float(A.y * inv);
+            o[2] = E::from_float(A.z * inv);
+            o[3] = E::from_float(A.w * inv);
             if (lane == 0) done[r] = 0;  // leave the counter ready for the next call
         }
     }
@@ -246,6 +298,8 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     int64_t W = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0) * 8;
     const int64_t cap = rows * (sparse_max_parts(rows, k) - 1);
     if (W > cap) W = cap;
+    // at most 32 parts per row: every part costs its row's merge a load
+    if (W > rows * 32) W = rows * 32;
     if (W > N) W = N;
     const int64_t grid = (W + 7) / 8;
     using T = typename E::T;

@@ -14,7 +14,13 @@
 
 namespace loki {
 
-constexpr int kTopkChunkTarget = 8192;  // keys per CTA the launcher aims for
+#ifndef LOKI_TOPK_CHUNK_TARGET
+#define LOKI_TOPK_CHUNK_TARGET 32768  // keys one CTA holds before a row is split over a cluster
+#endif
+#ifndef LOKI_TOPK_SPLIT_FEW_ROWS
+#define LOKI_TOPK_SPLIT_FEW_ROWS 0    // also split rows when they are fewer than 2 per SM
+#endif
+constexpr int kTopkChunkTarget = LOKI_TOPK_CHUNK_TARGET;
 
 // One CTA (or one cluster of CTAs) per row. CTA rank r of the row's cluster
 // holds keys [r * chunk, min((r + 1) * chunk, S)); chunk is a multiple of 4
@@ -221,10 +227,11 @@ bool topk_shape(int64_t rows, int64_t S, int sm_count, int* C_out, int* chunk_ou
                 int* gi_out) {
     int C = 1;
     auto chunk_of = [&](int c) { return (int)(((S + c - 1) / c + 3) / 4 * 4); };
-    // split a row while its CTA would hold more than the target, or while
-    // there are fewer than two CTAs per SM and the halves keep >= 1024 keys
+    // split a row over a cluster only while its CTA would hold more than the
+    // target (measured: one CTA per row beats a cluster at 4096 and 32768 keys)
     while (C < kTkMaxCluster &&
-           (chunk_of(C) > kTopkChunkTarget || (rows * C < 2 * sm_count && chunk_of(2 * C) >= 1024)))
+           (chunk_of(C) > kTopkChunkTarget ||
+            (LOKI_TOPK_SPLIT_FEW_ROWS && rows * C < 2 * sm_count && chunk_of(2 * C) >= 1024)))
         C *= 2;
     const int chunk = chunk_of(C);
     // 128 threads up to 2048 keys, then 256 threads with up to 8 groups of 4
