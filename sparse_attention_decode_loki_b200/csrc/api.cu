@@ -327,14 +327,15 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
     float* scores = at<float>(ws, w.scores);
     int* done = at<int>(ws, w.done);
     const int rows = B * H_q;
-    // Four kernels. Over a low-dim key plane: the TMA-staged score scan,
-    // which rotates the queries' first d_lo columns itself and streams keys
-    // at once, with the full query projection (which also zeroes the
-    // attention kernel's row counters) launched beside it; over the row
-    // layout: the projection, then the register-staged scan. Then top-k and
-    // attention with its row merge. The first kernel is ordered normally
-    // after whatever precedes the call; the second and top-k use programmatic
-    // dependent launch.
+    // Over a low-dim key plane: the TMA-staged score scan, which rotates the
+    // queries' first d_lo columns itself and streams keys at once, with the
+    // full query projection (which also zeroes the attention kernel's row
+    // counters) launched beside it; over the row layout: the projection,
+    // then the register-staged scan. Then selection and attention: one
+    // persistent kernel for small decodes, else top-k followed by attention
+    // with its row merge. The first kernel is ordered normally
+    // after whatever precedes the call; the rest use programmatic dependent
+    // launch.
     const bool fused = Kt_lo != nullptr && loki::score_plane_fuses(t, H_q / H_kv, d_lo, D);
     if (fused) {
         LOKI_CUDA(loki::launch_score_plane(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
@@ -354,9 +355,16 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                                                 d, scores, s, true),
                       name);
     }
+    if (loki::select_attend_fits(t, (int64_t)rows, S, D, k)) {
+        // small decode: selection and attention in one persistent kernel
+        LOKI_CUDA(loki::launch_select_attend(t, scores, q_rot, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                             S_max, k, resolve_scale(scale, D), out, selected_idx,
+                                             s, true),
+                  name);
+        return LOKI_OK;
+    }
     LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
-    // attention is a programmatic dependent of top-k too: its CTAs set up
-    // their copy pipeline as SMs drain and wait for the selection
+    // attention is a programmatic dependent of top-k too
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,

@@ -73,6 +73,17 @@ cudaError_t launch_decode_fused(Dt dt, const void* q, const float* P, const void
                                 int64_t S_max, int d_lo, int d, int64_t k, float scale, void* out,
                                 int32_t* sel, cudaStream_t s);
 
+// Whether the decode takes the one-kernel selection + attention: small
+// decodes (rows * k <= 8192, rows of at most 8192 keys, head dim 128).
+bool select_attend_fits(Dt dt, int64_t rows, int64_t S, int D, int64_t k);
+// Top-k of every (batch, query head) row of `scores` [B * H_q, S] and exact
+// attention over the selected tokens, in one kernel: writes sel [B * H_q, k]
+// and out [B * H_q, 128]. q_rot is q~ [B * H_q, 128] fp32.
+cudaError_t launch_select_attend(Dt dt, const float* scores, const float* q_rot, const void* Kt,
+                                 const void* V, int B, int H_q, int H_kv, int64_t S,
+                                 int64_t S_max, int64_t k, float scale, void* out, int32_t* sel,
+                                 cudaStream_t s, bool pdl);
+
 // partial slots per (batch, query head) row of the sparse attention split
 int64_t sparse_max_parts(int64_t rows, int64_t k);
 // done[B*H_q] must be zero on entry (per-row completion counters; the last

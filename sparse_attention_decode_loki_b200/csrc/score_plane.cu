@@ -29,7 +29,13 @@ constexpr int kScoreConsumers = kScoreConsumerWarps * 32;
 constexpr int kScoreThreads = kScoreConsumers + 32;
 // one CTA per SM (9 warps at ~104 registers leave no room for a second);
 // a 192 KB ring measured no faster than this one
-constexpr int kScoreRingBytes = 96 * 1024;
+#ifndef LOKI_SCORE_RING_KB
+#define LOKI_SCORE_RING_KB 96
+#endif
+#ifndef LOKI_SCORE_MINB
+#define LOKI_SCORE_MINB 1
+#endif
+constexpr int kScoreRingBytes = LOKI_SCORE_RING_KB * 1024;
 constexpr int kScoreMaxStages = 16;
 
 // NV = 16-byte chunks per plane row (d_lo * elem / 16). A tile is 256 rows,
@@ -42,7 +48,7 @@ constexpr int kScoreMaxStages = 16;
 // ahead, and the per-part partial sums meet in shared memory. Without it the
 // consumers read q~ from q_rot after the preceding kernel completes.
 template <class E, int G, int NV, bool kFuseQ>
-__global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
+__global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
     const float* __restrict__ P, const typename E::T* __restrict__ Klo,
     float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,

@@ -164,9 +164,19 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
         for (int cb = j0; cb < j1; cb += kWarpIdx) {
             const int n = min(kWarpIdx, j1 - cb);
             __syncwarp();
-            for (int t = lane; t < n; t += 32) {
-                const int tok = __ldg(ip + cb + t);
-                widx[t] = ((unsigned)tok < (unsigned)S) ? tok : -1;
+            {
+                // all of a lane's indices in flight at once (n <= 256 = 8 x 32)
+                int tk[kWarpIdx / 32];
+#pragma unroll
+                for (int u = 0; u < kWarpIdx / 32; ++u) {
+                    const int t = lane + 32 * u;
+                    tk[u] = t < n ? __ldg(ip + cb + t) : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < kWarpIdx / 32; ++u) {
+                    const int t = lane + 32 * u;
+                    if (t < n) widx[t] = ((unsigned)tk[u] < (unsigned)S) ? tk[u] : -1;
+                }
             }
             __syncwarp();
 #if LOKI_SP_PIPE

@@ -215,7 +215,9 @@ static cudaError_t launch_shape(int nt, int gi, const float* scores, int64_t row
 #define LOKI_TK(NT_, I_) \
     if (nt == NT_ && gi == I_) return launch_rows<NT_, I_, kCl>(scores, rows, S, k, C, chunk, idx, s, pdl);
     LOKI_TK(128, 1) LOKI_TK(128, 2) LOKI_TK(128, 4)
-    LOKI_TK(256, 4) LOKI_TK(256, 8) LOKI_TK(512, 8) LOKI_TK(1024, 8)
+    LOKI_TK(256, 4) LOKI_TK(256, 8) LOKI_TK(512, 8)
+    LOKI_TK(256, 1) LOKI_TK(512, 1)
+    LOKI_TK(1024, 1) LOKI_TK(1024, 2) LOKI_TK(1024, 4) LOKI_TK(1024, 8)
 #undef LOKI_TK
     return cudaErrorInvalidValue;
 }
@@ -236,7 +238,15 @@ bool topk_shape(int64_t rows, int64_t S, int sm_count, int* C_out, int* chunk_ou
     const int chunk = chunk_of(C);
     // 128 threads up to 2048 keys, then 256 threads with up to 8 groups of 4
     // keys each, then more threads (measured: 256 x 4 beats 128 x 8 at 4096)
+    // Many rows (at least two CTAs per SM): 128 threads up to 2048 keys, then
+    // 256 threads with up to 8 groups of 4 keys each (measured: 256 x 4 beats
+    // 128 x 8 at 4096 keys), then more threads. Few rows: one group of 4 keys
+    // per thread up to 1024 threads (measured: 1024 x 1 takes two thirds of
+    // the 256 x 4 time at 32 rows of 4096 keys).
+    const bool few = rows * C < 2 * sm_count;
     int nt = chunk > 2048 ? 256 : 128, gi = 1;
+    if (few)
+        while (nt < 1024 && 4 * nt < chunk) nt *= 2;  // one group of 4 keys per thread
     while (4 * nt * gi < chunk && gi < 8) gi *= 2;
     while (4 * nt * gi < chunk && nt < 1024) nt *= 2;
     if (4 * nt * gi < chunk) return false;

@@ -82,10 +82,17 @@ __device__ __forceinline__ void tk_zero(const TkSmem& sm) {
         reinterpret_cast<uint4*>(sm.hist1)[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
-// The CTA's place in its cluster (rank 0 of 1 without one).
-template <bool kCl>
+// The CTA's place in its cluster (rank 0 of 1 without one), and the block
+// barrier of the selecting threads: __syncthreads() (kBar = 0), or named
+// barrier kBar over the first kBarThreads threads of the block when the
+// selection runs on a subset of its warps.
+template <bool kCl, int kBar = 0, int kBarThreads = 0>
 struct TkCluster {
     int rank = 0, size = 1;
+    __device__ __forceinline__ void bsync() const {
+        if constexpr (kBar == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"n"(kBar), "n"(kBarThreads) : "memory");
+    }
     __device__ __forceinline__ void init() {
         if constexpr (kCl) {
             cg::cluster_group c = cg::this_cluster();
@@ -95,7 +102,7 @@ struct TkCluster {
     }
     __device__ __forceinline__ void sync() const {
         if constexpr (kCl) cg::this_cluster().sync();
-        else __syncthreads();
+        else bsync();
     }
     // the copy of a shared-memory object in the CTA of rank r
     template <class T>
@@ -133,12 +140,12 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
 
 // Sum of v over all warps before this one (and over all warps), through
 // red[0, NW); ends with every thread past one block barrier.
-template <int NT>
-__device__ __forceinline__ int block_warp_prefix(int v, int* red, int* all) {
+template <int NT, class CL>
+__device__ __forceinline__ int block_warp_prefix(const CL& cl, int v, int* red, int* all) {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) red[warp] = v;
-    __syncthreads();
+    cl.bsync();
     int lo = (lane < warp) ? red[lane] : 0;
     int tot = (lane < NW) ? red[lane] : 0;
 #pragma unroll
@@ -156,9 +163,8 @@ __device__ __forceinline__ int block_warp_prefix(int v, int* red, int* all) {
 // registers. The bin, the rank left inside it and its cluster count go to
 // red[] and are valid for every thread on return. The caller has made every
 // copy of hist complete and visible (block or cluster barrier).
-template <int NT, int NB, bool kCl>
-__device__ __forceinline__ void tk_find_bin(const TkCluster<kCl>& cl, const uint32_t* hist, int krem,
-                                            int* red) {
+template <int NT, int NB, bool kCl, class CL>
+__device__ __forceinline__ void tk_find_bin(const CL& cl, const uint32_t* hist, int krem, int* red) {
     constexpr int PER = NB / NT;  // 1..16
     static_assert(PER >= 1 && NB % NT == 0, "bins per thread");
     constexpr int NW = NT / 32;
@@ -193,7 +199,7 @@ __device__ __forceinline__ void tk_find_bin(const TkCluster<kCl>& cl, const uint
     int wtot;
     const int in_warp_above = warp_suffix_excl(local, &wtot);
     if (lane == 0) red[warp] = wtot;
-    __syncthreads();
+    cl.bsync();
     int hi = (lane > warp && lane < NW) ? red[lane] : 0;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) hi += __shfl_xor_sync(0xffffffffu, hi, off);
@@ -213,7 +219,7 @@ __device__ __forceinline__ void tk_find_bin(const TkCluster<kCl>& cl, const uint
             cum += (int)c[e];
         }
     }
-    __syncthreads();
+    cl.bsync();
 }
 
 // Selects the k largest keys of a row and writes their global indices in
@@ -227,15 +233,17 @@ __device__ __forceinline__ void tk_find_bin(const TkCluster<kCl>& cl, const uint
 // Every thread of every CTA of the cluster must call it. On return every
 // thread is past its last barrier (in a cluster: past a final cluster
 // barrier, so no CTA's shared memory is still read by another).
-template <int NT, int I, bool kCl>
-__device__ __forceinline__ void tk_select(const TkCluster<kCl>& cl, const uint4 (&v)[I], int base,
-                                          int k, int32_t* out, const TkSmem& sm) {
+template <int NT, int I, bool kCl, int kBar = 0>
+__device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT : 0)>& cl,
+                                          const uint4 (&v)[I], int base, int k, int32_t* out,
+                                          const TkSmem& sm) {
+    using CL = TkCluster<kCl, kBar, (kBar ? NT : 0)>;
     static_assert(I == 1 || I == 2 || I == 4 || I == 8, "groups per thread");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int* red = sm.red;
     // every CTA's pass-1 histogram is complete
     cl.sync();
-    tk_find_bin<NT, kTkBins1, kCl>(cl, sm.hist1, k, red);
+    tk_find_bin<NT, kTkBins1, kCl, CL>(cl, sm.hist1, k, red);
     const uint32_t bin1 = (uint32_t)red[kRedBin];
     int krem = red[kRedKrem];
     // pass 2: bits 20..10 of the keys in the threshold bin
@@ -247,7 +255,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl>& cl, const uint4 
             if (kk[e] != 0u && (kk[e] >> 21) == bin1) atomicAdd(&sm.hist2[(kk[e] >> 10) & 2047u], 1u);
     }
     cl.sync();
-    tk_find_bin<NT, kTkBins2, kCl>(cl, sm.hist2, krem, red);
+    tk_find_bin<NT, kTkBins2, kCl, CL>(cl, sm.hist2, krem, red);
     const uint32_t pre = (bin1 << 11) | (uint32_t)red[kRedBin];
     krem = red[kRedKrem];
     // pass 3: bits 9..0 of the keys sharing the 22-bit prefix
@@ -259,7 +267,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl>& cl, const uint4 
             if (kk[e] != 0u && (kk[e] >> 10) == pre) atomicAdd(&sm.hist3[kk[e] & 1023u], 1u);
     }
     cl.sync();
-    tk_find_bin<NT, kTkBins3, kCl>(cl, sm.hist3, krem, red);
+    tk_find_bin<NT, kTkBins3, kCl, CL>(cl, sm.hist3, krem, red);
     const uint32_t T = (pre << 10) | (uint32_t)red[kRedBin];
     const int take_T = red[kRedKrem];  // keys equal to T in the set (the lowest-index ones)
     const int cnt_T = red[kRedCnt];    // keys equal to T in the row
@@ -321,7 +329,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl>& cl, const uint4 
         int epos[I];
         const int wtot = warp_positions(eqm, epos);
         int all;
-        const int wpre = block_warp_prefix<NT>(wtot, red, &all);
+        const int wpre = block_warp_prefix<NT>(cl, wtot, red, &all);
         const int before = wpre + cluster_prefix(all, kRedTotal);
         uint32_t keep = 0u;
 #pragma unroll
@@ -336,12 +344,12 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl>& cl, const uint4 
                 }
         }
         sel = gtm | keep;
-        __syncthreads();  // red[0, NW) is reused below
+        cl.bsync();  // red[0, NW) is reused below
     }
     int spos[I];
     const int wtot = warp_positions(sel, spos);
     int all;
-    const int wpre = block_warp_prefix<NT>(wtot, red, &all);
+    const int wpre = block_warp_prefix<NT>(cl, wtot, red, &all);
     const int before = wpre + cluster_prefix(all, kRedTotal + 1);
     const int gw = warp * 32 * I + lane;
 #pragma unroll

@@ -55,7 +55,7 @@ def _threads():
     return workloads._threads(None)
 
 
-@functools.lru_cache(maxsize=4)
+@functools.lru_cache(maxsize=3)
 def host_inputs(wl: workloads.Workload) -> HostInputs:
     g = workloads.generate(wl)
     Ps, eigs = [], []

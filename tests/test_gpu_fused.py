@@ -56,6 +56,7 @@ CASES = [
     # name, workload, overrides, d_lo, S_max
     ("tiny-f32", "tiny", {}, 32, 300),
     ("llama2-7b", "llama2-7b", {}, 32, None),
+    ("llama2-13b", "llama2-13b", {}, 32, None),
     ("ragged-S-d20", "llama2-7b", dict(B=2, H_q=2, H_kv=2, S=1000, d=20, k=77), 32, 1024),
     ("k1", "llama2-7b", dict(B=1, H_q=2, H_kv=2, S=513, k=1), 32, 600),
     ("k-all", "llama2-7b", dict(B=1, H_q=2, H_kv=2, S=300, k=300), 32, 300),

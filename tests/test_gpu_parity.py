@@ -157,52 +157,25 @@ def test_all_dims_all_tokens_is_dense(loki, cuda):
 
 
 # ---------------------------------------------------------------------------
-# large workloads: full launch, sampled rows
+# large workloads
 # ---------------------------------------------------------------------------
 
-def sampled_run(loki, dev, wl, n_rows, seed=7, plane=False):
-    """Full-size launch; the sampled rows' blocks hold generator + oracle bytes,
-    every other block holds seeded random filler (its rows are not checked)."""
-    torch = _torch()
-    rows = workloads.sample_rows(wl, n_rows, seed)
-    need_kv = sorted({h // wl.G for _, h in rows})
-    Rs = {h: workloads.rotation(wl, h) for h in need_kv}
-    P = np.tile(np.eye(wl.D, dtype=np.float32), (wl.H_kv, 1, 1))
-    for h in need_kv:
-        Pm, _ = oracle.calibrate_pca(workloads.calibration_keys(wl, h, Rs[h]))
-        P[h] = Pm.astype(np.float32)
-    dt = parity.torch_dtype(wl)
-    g = torch.Generator(device=dev)
-    g.manual_seed(wl.seed)
-    Kt = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
-    V = torch.randn((wl.B, wl.H_kv, wl.S, wl.D), generator=g, device=dev, dtype=dt)
-    q = torch.randn((wl.B, wl.H_q, wl.D), generator=g, device=dev, dtype=dt)
-    host = {}
-    for b, h in rows:
-        hk = h // wl.G
-        if (b, hk) not in host:
-            K = workloads.keys_block(wl, b, hk, Rs[hk])
-            Vb = workloads.values_block(wl, b, hk)
-            Ktb = oracle.rotate_keys(K, P[hk].astype(np.float64), wl.dtype).astype(np.float32)
-            host[(b, hk)] = (Ktb, Vb)
-            Kt[b, hk] = torch.from_numpy(Ktb).to(dev).to(dt)
-            V[b, hk] = torch.from_numpy(Vb).to(dev).to(dt)
-        q[b, h] = torch.from_numpy(workloads.query_vec(wl, b, h, Rs[hk])).to(dev).to(dt)
-    Pt = torch.from_numpy(P).to(dev)
-    Kt_lo = Kt[..., : wl.d].contiguous() if plane else None
-    out, idx = loki.loki_decode_attention(q, Kt, V, Pt, wl.S, wl.d, wl.k, wl.scale, Kt_lo=Kt_lo)
-    out = out.float().cpu().numpy()
-    idx = idx.cpu().numpy()
-    qh = q.float().cpu().numpy()
-    assert loki.loki_device_error(reset=True) == 0, "a staged kernel's bounded wait gave up"
-    checks = []
-    for b, h in rows:
-        hk = h // wl.G
-        Ktb, Vb = host[(b, hk)]
-        checks.append(_check_block(wl, P[hk], qh[b, h], Ktb, Vb, idx[b, h], out[b, h], (b, h)))
-    del Kt, V
-    torch.cuda.empty_cache()
-    return parity.summarize(checks)
+@pytest.mark.parametrize("plane", [False, True])
+def test_llama2_13b_every_row(loki, cuda, plane):
+    """The benchmark's workload and launch configuration, every (batch, head)
+    row against the oracle."""
+    inp = parity.host_inputs(workloads.get("llama2-13b"))
+    res = run_full(loki, inp, cuda, d_lo=32 if plane else None)
+    s = check_all_rows(inp, res)
+    assert s["rows"] == 640
+
+
+@pytest.mark.parametrize("plane", [False, True])
+def test_llama3_8b_gqa_every_row(loki, cuda, plane):
+    inp = parity.host_inputs(workloads.get("llama3-8b-gqa"))
+    res = run_full(loki, inp, cuda, d_lo=16 if plane else None)
+    s = check_all_rows(inp, res)
+    assert s["rows"] == 128
 
 
 def _check_block(wl, P, q, Kt, V, gidx, gout, row):
@@ -212,27 +185,81 @@ def _check_block(wl, P, q, Kt, V, gidx, gout, row):
     return parity.check_row(inp, 0, 0, gidx, gout, wl.d, wl.k, wl.scale)
 
 
-@pytest.mark.parametrize("plane", [False, True])
-def test_llama2_13b_sampled(loki, cuda, plane):
-    s = sampled_run(loki, cuda, workloads.get("llama2-13b"), 24, plane=plane)
-    assert s["rows"] == 24
+def _sweep_group(B, S):
+    return [p for p in workloads.sweep_points() if p.B == B and p.S == S]
 
 
-@pytest.mark.parametrize("plane", [False, True])
-def test_llama3_8b_gqa_sampled(loki, cuda, plane):
-    s = sampled_run(loki, cuda, workloads.get("llama3-8b-gqa"), 16, plane=plane)
-    assert s["rows"] == 16
+SWEEP_GROUPS = sorted({(p.B, p.S) for p in workloads.sweep_points()})
 
 
-SWEEP_SAMPLE = ["sweep-B1-S2048-d16-k1of8", "sweep-B8-S16384-d32-k1of4",
-                "sweep-B1-S131072-d64-k1of8", "sweep-B64-S2048-d64-k1of4",
-                "sweep-B8-S131072-d16-k1of4"]
-
-
-@pytest.mark.parametrize("name", SWEEP_SAMPLE)
-def test_sweep_sampled(loki, cuda, name):
-    s = sampled_run(loki, cuda, workloads.get(name), 6, plane=True)
-    assert s["rows"] == 6
+@pytest.mark.parametrize("B,S", SWEEP_GROUPS, ids=[f"B{b}-S{s}" for b, s in SWEEP_GROUPS])
+def test_sweep_every_point_sampled_rows(loki, cuda, B, S):
+    """All six (d, k/S) points of one (B, S) of the sweep at full size, in the
+    benchmark's layout (a key plane of d columns; the row layout where the
+    plane does not fit the device). The points share their inputs (one seed),
+    so the cache is filled once per (B, S): random filler everywhere and
+    generator bytes in the blocks of 6 sampled rows, which are checked against
+    the oracle."""
+    torch = _torch()
+    pts = _sweep_group(B, S)
+    wl = pts[0]
+    e = wl.elem_bytes
+    kv_bytes = 2 * e * B * wl.H_kv * S * wl.D
+    scores_bytes = 4 * B * wl.H_q * S
+    margin = 3 << 30
+    free, _ = torch.cuda.mem_get_info(cuda)
+    if kv_bytes + scores_bytes + margin > free:
+        pytest.skip(f"B={B}, S={S}: the cache ({kv_bytes / 1e9:.1f} GB) does not fit "
+                    f"the free device memory ({free / 1e9:.1f} GB)")
+    rows = workloads.sample_rows(wl, 6, 7)
+    need_kv = sorted({h // wl.G for _, h in rows})
+    Rs = {h: workloads.rotation(wl, h) for h in need_kv}
+    P = np.tile(np.eye(wl.D, dtype=np.float32), (wl.H_kv, 1, 1))
+    for h in need_kv:
+        Pm, _ = oracle.calibrate_pca(workloads.calibration_keys(wl, h, Rs[h]))
+        P[h] = Pm.astype(np.float32)
+    dt = parity.torch_dtype(wl)
+    g = torch.Generator(device=cuda)
+    g.manual_seed(wl.seed + B + S)
+    Kt = torch.randn((B, wl.H_kv, S, wl.D), generator=g, device=cuda, dtype=dt)
+    V = torch.randn((B, wl.H_kv, S, wl.D), generator=g, device=cuda, dtype=dt)
+    q = torch.randn((B, wl.H_q, wl.D), generator=g, device=cuda, dtype=dt)
+    host = {}
+    for b, h in rows:
+        hk = h // wl.G
+        if (b, hk) not in host:
+            K = workloads.keys_block(wl, b, hk, Rs[hk])
+            Vb = workloads.values_block(wl, b, hk)
+            Ktb = oracle.rotate_keys(K, P[hk].astype(np.float64), wl.dtype).astype(np.float32)
+            host[(b, hk)] = (Ktb, Vb)
+            Kt[b, hk] = torch.from_numpy(Ktb).to(cuda).to(dt)
+            V[b, hk] = torch.from_numpy(Vb).to(cuda).to(dt)
+        q[b, h] = torch.from_numpy(workloads.query_vec(wl, b, h, Rs[hk])).to(cuda).to(dt)
+    Pt = torch.from_numpy(P).to(cuda)
+    qh = q.float().cpu().numpy()
+    layouts = {}
+    for pt in pts:
+        free, _ = torch.cuda.mem_get_info(cuda)
+        plane_bytes = e * B * wl.H_kv * S * pt.d
+        Kt_lo = None
+        if plane_bytes + scores_bytes + margin <= free:
+            Kt_lo = Kt[..., : pt.d].contiguous()
+        out, idx = loki.loki_decode_attention(q, Kt, V, Pt, S, pt.d, pt.k, pt.scale, Kt_lo=Kt_lo)
+        out = out.float().cpu().numpy()
+        idx = idx.cpu().numpy()
+        assert loki.loki_device_error(reset=True) == 0, "a staged kernel's bounded wait gave up"
+        layouts[pt.name] = "plane" if Kt_lo is not None else "rows"
+        del Kt_lo
+        checks = []
+        for b, h in rows:
+            hk = h // wl.G
+            Ktb, Vb = host[(b, hk)]
+            checks.append(_check_block(pt, P[hk], qh[b, h], Ktb, Vb, idx[b, h], out[b, h], (b, h)))
+        assert parity.summarize(checks)["rows"] == 6
+        torch.cuda.empty_cache()
+    print(f"sweep B={B} S={S}: layouts {layouts}")
+    del Kt, V
+    torch.cuda.empty_cache()
 
 
 # ---------------------------------------------------------------------------
