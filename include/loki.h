@@ -169,6 +169,31 @@ LOKI_API loki_status loki_decode_attention_plane(const void* q, const void* Kt_c
                                                  void* stream);
 
 /*
+ * One decode step that first appends the step's new tokens: the poster page's
+ * "Loki's Computational Cost" section names the per-step KV-cache append as a
+ * limiting cost, so here it is folded into the step's first kernel instead of
+ * running as a launch of its own.
+ *   K_new, V_new [B, H_kv, T, D] (dt): the T new tokens of every (batch, KV
+ *           head); their rotated keys K~ = K_new P (fp32 accumulate, rounded
+ *           to dt, exactly as loki_append_keys) go to cache rows [pos, pos + T)
+ *           of Kt_cache (and of the plane Kt_lo when it is not NULL: d_lo
+ *           columns, as loki_append_keys_plane), their values to V_cache.
+ *   Then the decode over S = pos + T cached tokens, as loki_decode_attention
+ *   (Kt_lo == NULL) or loki_decode_attention_plane: same arguments, same
+ *   results, same workspace size (loki_decode_workspace_size with S).
+ * The query rotation and the key rotation run in one kernel; the score scan
+ * starts streaming rows [0, pos) at once and waits for that kernel only
+ * before reading the new rows.
+ *   requires 1 <= T, 0 <= pos, pos + T <= S_max, 1 <= k <= pos + T
+ */
+LOKI_API loki_status loki_decode_step(const void* q, const void* K_new, const void* V_new,
+                                      const float* P, void* Kt_cache, void* V_cache, void* Kt_lo,
+                                      int d_lo, int B, int H_q, int H_kv, int T, int64_t pos,
+                                      int64_t S_max, int D, int d, int64_t k, float scale,
+                                      loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/*
  * The same decode step as loki_decode_attention_plane in a single kernel:
  * one thread block per (batch, KV head) unit rotates the unit's queries,
  * scans its key plane, keeps the scores in on-chip shared memory, selects the

@@ -23,6 +23,7 @@ __all__ = [
     "LokiError", "LIB_PATH",
     "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
     "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_fused",
+    "loki_decode_step",
     "loki_decode_attention_noalloc",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
@@ -229,6 +230,46 @@ def loki_decode_attention_plane(q, Kt_cache, V_cache, Kt_lo, P, S: int, d: int, 
     """loki_decode_attention scoring from the low-dimensional key plane Kt_lo."""
     return loki_decode_attention(q, Kt_cache, V_cache, P, S, d, k, scale, out, selected_idx,
                                  workspace, Kt_lo=Kt_lo)
+
+
+def loki_decode_step(q: torch.Tensor, K_new: torch.Tensor, V_new: torch.Tensor, P: torch.Tensor,
+                     Kt_cache: torch.Tensor, V_cache: torch.Tensor, pos: int, d: int, k: int,
+                     scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                     selected_idx: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     Kt_lo: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Append K_new, V_new [B, H_kv, T, D] at cache rows [pos, pos + T) (keys
+    rotated by P; also into the key plane Kt_lo when given), then decode over
+    the pos + T cached tokens. Returns (out, selected_idx) as loki_decode_attention."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q, Kt_cache, V_cache, P)
+    _cuda(q, K_new, V_new)
+    if K_new.dim() != 4 or K_new.shape[:2] != (B, H_kv) or K_new.shape[3] != D:
+        raise ValueError("K_new must be [B, H_kv, T, D]")
+    if V_new.shape != K_new.shape or K_new.dtype != q.dtype or V_new.dtype != q.dtype:
+        raise ValueError("V_new must match K_new, with the caches' dtype")
+    T = K_new.shape[2]
+    S = pos + T
+    if out is None:
+        out = torch.empty_like(q)
+    if selected_idx is None:
+        selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    _cuda(q, out, selected_idx)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    if S > S_max:
+        raise ValueError("pos + T must be <= S_max")
+    d_lo = 0
+    if Kt_lo is not None:
+        _check_plane(Kt_lo, Kt_cache)
+        d_lo = Kt_lo.shape[3]
+    ws = _ws(loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k), dev, workspace)
+    check(lib.loki_decode_step(q.data_ptr(), K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+                               Kt_cache.data_ptr(), V_cache.data_ptr(),
+                               Kt_lo.data_ptr() if Kt_lo is not None else None, d_lo, B, H_q,
+                               H_kv, T, pos, S_max, D, d, k, float(scale), _dt(q), out.data_ptr(),
+                               selected_idx.data_ptr(), ws.data_ptr(), _ws_bytes(ws),
+                               _stream(dev)), "loki_decode_step")
+    return out, selected_idx
 
 
 def loki_decode_attention_fused(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,

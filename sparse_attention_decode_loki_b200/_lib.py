@@ -42,6 +42,10 @@ PROTOTYPES = {
                                             c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,
                                             c_int, c_int64, c_float, c_int, c_void_p, c_void_p,
                                             c_void_p, c_size_t, c_void_p]),
+    "loki_decode_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                 c_void_p, c_int, c_int, c_int, c_int, c_int, c_int64, c_int64,
+                                 c_int, c_int, c_int64, c_float, c_int, c_void_p, c_void_p,
+                                 c_void_p, c_size_t, c_void_p]),
     "loki_decode_attention_fused": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                             c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,
                                             c_int, c_int64, c_float, c_int, c_void_p, c_void_p,

@@ -287,12 +287,40 @@ static loki_status check_decode_common(int B, int H_q, int H_kv, int64_t S, int6
     return LOKI_OK;
 }
 
+// Selection and attention after the score scan (both programmatic dependents).
+static loki_status decode_tail(const char* name, loki::Dt t, float* scores, float* q_rot,
+                               int* done, void* ws, const DecodeWs& w, const void* Kt_cache,
+                               const void* V_cache, int B, int H_q, int H_kv, int64_t S,
+                               int64_t S_max, int D, int64_t k, float scale, void* out,
+                               int32_t* selected_idx, cudaStream_t s) {
+    const int rows = B * H_q;
+    if (loki::select_attend_fits(t, (int64_t)rows, S, D, k)) {
+        // small decode: selection and attention in one persistent kernel
+        LOKI_CUDA(loki::launch_select_attend(t, scores, q_rot, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                             S_max, k, resolve_scale(scale, D), out, selected_idx,
+                                             s, true),
+                  name);
+        return LOKI_OK;
+    }
+    LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
+    // attention is a programmatic dependent of top-k too
+    LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
+                                            S, S_max, D, k, resolve_scale(scale, D), out,
+                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
+                                            true),
+              name);
+    return LOKI_OK;
+}
+
+// One decode step; with K_new (T new tokens per (batch, KV head)) the step
+// first appends them at cache rows [S - T, S), rotated, in its first kernel.
 static loki_status decode_impl(const char* name, const void* q, const void* Kt_cache,
                                const void* V_cache, const void* Kt_lo, int d_lo, const float* P,
                                int B, int H_q, int H_kv, int64_t S, int64_t S_max, int D, int d,
                                int64_t k, float scale, loki_dtype dt, void* out,
-                               int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream) {
-    g_last_error.clear();
+                               int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream,
+                               const void* K_new = nullptr, const void* V_new = nullptr,
+                               int T = 0) {
     LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
     LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
     LOKI_REQUIRE(k >= 1 && k <= S, LOKI_ERR_INVALID_ARG, "k must be in [1, S] (got %lld)",
@@ -309,11 +337,45 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
         LOKI_PTR(Kt_lo, 16);
         LOKI_REQUIRE(d <= d_lo, LOKI_ERR_INVALID_ARG, "d (%d) must be <= d_lo (%d)", d, d_lo);
     }
+    if (K_new != nullptr) {
+        LOKI_PTR(K_new, 16);
+        LOKI_PTR(V_new, 16);
+        LOKI_REQUIRE(T >= 1 && T <= S, LOKI_ERR_INVALID_ARG,
+                     "T must be in [1, S] new tokens (got %d)", T);
+    }
     const DecodeWs w = decode_ws(B, H_q, S, D, k);
     LOKI_REQUIRE(ws_bytes >= w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
                  "workspace %zu bytes < required %zu", ws_bytes, w.total);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const loki::Dt t = to_dt(dt);
+    float* q_rot = at<float>(ws, w.q_rot);
+    float* scores = at<float>(ws, w.scores);
+    int* done = at<int>(ws, w.done);
+    const int rows = B * H_q;
+    if (K_new != nullptr) {
+        // Append and decode: the first kernel rotates the queries and the new
+        // keys (writing their cache, plane and value rows); the score scan is
+        // its programmatic dependent and streams the older rows at once,
+        // waiting for it only before the tiles that hold the new rows.
+        const int64_t pos = S - T;
+        LOKI_CUDA(loki::launch_rotate(t, q, K_new, V_new, P, q_rot, const_cast<void*>(Kt_cache),
+                                      const_cast<void*>(V_cache), const_cast<void*>(Kt_lo), d_lo,
+                                      B, H_q, H_kv, T, D, S_max, pos, s, done, rows, false),
+                  name);
+        if (Kt_lo != nullptr) {
+            const bool fuse = loki::score_plane_fuses(t, H_q / H_kv, d_lo, D);
+            LOKI_CUDA(loki::launch_score_plane(t, q_rot, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
+                                               scores, s, true, fuse ? q : nullptr,
+                                               fuse ? P : nullptr, pos),
+                      name);
+        } else {
+            LOKI_CUDA(loki::launch_score_lowdim(t, q_rot, Kt_cache, B, H_q, H_kv, S, S_max, D, D,
+                                                d, scores, s, true),
+                      name);
+        }
+        return decode_tail(name, t, scores, q_rot, done, ws, w, Kt_cache, V_cache, B, H_q, H_kv,
+                           S, S_max, D, k, scale, out, selected_idx, s);
+    }
     // Many (batch, KV head) units over a low-dim key plane: one kernel does
     // the whole step per unit, with the scores in shared memory.
     if (Kt_lo != nullptr && loki::decode_fused_preferred(t, B, H_q, H_kv, S, D, d_lo, k)) {
@@ -323,10 +385,6 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                   name);
         return LOKI_OK;
     }
-    float* q_rot = at<float>(ws, w.q_rot);
-    float* scores = at<float>(ws, w.scores);
-    int* done = at<int>(ws, w.done);
-    const int rows = B * H_q;
     // Over a low-dim key plane: the TMA-staged score scan, which rotates the
     // queries' first d_lo columns itself and streams keys at once, with the
     // full query projection (which also zeroes the attention kernel's row
@@ -355,22 +413,8 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                                                 d, scores, s, true),
                       name);
     }
-    if (loki::select_attend_fits(t, (int64_t)rows, S, D, k)) {
-        // small decode: selection and attention in one persistent kernel
-        LOKI_CUDA(loki::launch_select_attend(t, scores, q_rot, Kt_cache, V_cache, B, H_q, H_kv, S,
-                                             S_max, k, resolve_scale(scale, D), out, selected_idx,
-                                             s, true),
-                  name);
-        return LOKI_OK;
-    }
-    LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S, k, selected_idx, s, true), name);
-    // attention is a programmatic dependent of top-k too
-    LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
-                                            S, S_max, D, k, resolve_scale(scale, D), out,
-                                            at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
-                                            true),
-              name);
-    return LOKI_OK;
+    return decode_tail(name, t, scores, q_rot, done, ws, w, Kt_cache, V_cache, B, H_q, H_kv, S,
+                       S_max, D, k, scale, out, selected_idx, s);
 }
 
 loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
@@ -395,6 +439,24 @@ loki_status loki_decode_attention_plane(const void* q, const void* Kt_cache, con
     return decode_impl("loki_decode_attention_plane", q, Kt_cache, V_cache, Kt_lo, d_lo, P, B,
                        H_q, H_kv, S, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes,
                        stream);
+}
+
+loki_status loki_decode_step(const void* q, const void* K_new, const void* V_new, const float* P,
+                             void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_q,
+                             int H_kv, int T, int64_t pos, int64_t S_max, int D, int d, int64_t k,
+                             float scale, loki_dtype dt, void* out, int32_t* selected_idx, void* ws,
+                             size_t ws_bytes, void* stream) {
+    if (K_new == nullptr || V_new == nullptr) {
+        g_last_error = "K_new and V_new must not be NULL";
+        return LOKI_ERR_INVALID_ARG;
+    }
+    if (pos < 0 || T < 1 || pos > kMaxS - T) {
+        g_last_error = "need pos >= 0, T >= 1 and pos + T < 2^31";
+        return LOKI_ERR_INVALID_ARG;
+    }
+    return decode_impl("loki_decode_step", q, Kt_cache, V_cache, Kt_lo, d_lo, P, B, H_q, H_kv,
+                       pos + T, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes, stream,
+                       K_new, V_new, T);
 }
 
 loki_status loki_decode_attention_fused(const void* q, const void* Kt_cache, const void* V_cache,

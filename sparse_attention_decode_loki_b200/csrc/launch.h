@@ -50,10 +50,13 @@ bool score_plane_fuses(Dt dt, int G, int d_lo, int D);
 // streams keys first and its consumers wait for q_rot. Given the raw queries
 // q and the bases P (head dim 128; score_plane_fuses) the consumers rotate the
 // query themselves, and the scan is launched without pdl whatever pdl says.
+// wait_row < S: rows [wait_row, S) of every unit are written by the preceding
+// kernel; the scan (launched as its programmatic dependent) streams the other
+// rows at once and waits for it before reading those.
 cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
                                int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
                                float* scores, cudaStream_t s, bool pdl, const void* q = nullptr,
-                               const float* P = nullptr);
+                               const float* P = nullptr, int64_t wait_row = INT64_MAX);
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
                         cudaStream_t s, bool pdl);
@@ -99,6 +102,17 @@ int64_t dense_max_parts(int64_t S);
 cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int B, int H_q,
                          int H_kv, int64_t S, int64_t S_max, int D, float scale, void* out,
                          float2* part_ml, float* part_acc, cudaStream_t s);
+
+// Rotation into the KV heads' PCA bases, in one kernel: the G query rows of
+// every (batch, KV head) into q_rot (q may be null), and T new keys per
+// (batch, KV head) into cache rows [pos, pos + T) of Kt_cache (and of the plane
+// Kt_lo when not null) with their values copied to V_cache (K_new may be
+// null). Also zeroes done[0, n_done). With pdl it is a programmatic dependent
+// of the preceding kernel that completes only after it (see the score scan).
+cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V_new,
+                          const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
+                          int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
+                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl);
 
 // ---- supporting subsystems -----------------------------------------------
 // Kt_lo (may be null): [B, H_kv, S_max, d_lo] plane that also receives the

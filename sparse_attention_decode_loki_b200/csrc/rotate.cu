@@ -1,0 +1,162 @@
+// Rotation of rows into a KV head's PCA basis: queries, q~ = q P, and new
+// keys appended to the KV-cache, K~ = K P (the key also goes to the
+// low-dimensional key plane; its value row is copied unchanged).
+//
+// Loki (NeurIPS 2024 poster page, "Visual Insights" Figure 1 caption: keys
+// and queries are used through their PCA projection; "Loki's Computational
+// Cost": keys are appended to the KV-cache at every decode step).
+//
+// One CTA per (KV head, block of 32 output columns, chunk of up to 32 rows of
+// that head): the 128 x 32 column block of P is staged once in shared memory
+// and used by every row of the chunk; each warp computes one row's 32 columns
+// per step, summing in fp32 in index order. A head's rows are, per sequence
+// b, its G query heads and then its T new keys; query rows go to q_rot
+// (fp32), key rows are rounded once to the cache type (nearest even) and
+// written at cache rows [pos, pos + T).
+#include "common.cuh"
+#include "launch.h"
+
+namespace loki {
+
+constexpr int kRotCols = 32;
+constexpr int kRotRows = 32;
+
+template <class E>
+__global__ void __launch_bounds__(256) k_rotate_rows(
+    const typename E::T* __restrict__ q, const typename E::T* __restrict__ K_new,
+    const typename E::T* __restrict__ V_new, const float* __restrict__ P, float* __restrict__ q_rot,
+    typename E::T* __restrict__ Kt_cache, typename E::T* __restrict__ V_cache,
+    typename E::T* __restrict__ Kt_lo, int d_lo, int B, int H_q, int H_kv, int G, int T, int D,
+    int64_t S_max, int64_t pos, int* __restrict__ done, int n_done, int hold) {
+    using Tp = typename E::T;
+    __shared__ float Ps[128][kRotCols];
+    __shared__ float xs[kRotRows][128];
+    // a programmatic dependent (the score scan) may start right away
+    griddep_launch_dependents();
+    // one-dimensional grid: CTA = (row chunk, column block, KV head), head fastest
+    const int64_t bid = blockIdx.x;
+    if (done != nullptr) {
+        const int64_t nb = gridDim.x;
+        for (int64_t i = bid * 256 + threadIdx.x; i < n_done; i += nb * 256) done[i] = 0;
+    }
+    const int ncb = (D + kRotCols - 1) / kRotCols;
+    const int hk = (int)(bid % H_kv);
+    const int cb = (int)((bid / H_kv) % ncb);
+    const int c0 = cb * kRotCols;
+    const int64_t r0 = (bid / H_kv / ncb) * kRotRows;
+    const int R = G + T;  // rows of the head per sequence
+    const int nrows = (int)min64(kRotRows, (int64_t)B * R - r0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float* Ph = P + (int64_t)hk * D * D;
+    // the P block: 128 rows x 32 columns = 1024 float4, 4 per thread, all in flight
+    float4 pv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int it = tid + u * 256;
+        const int i = it >> 3, c4 = (it & 7) * 4;
+        pv[u] = (i < D && c0 + c4 < D)
+                    ? __ldg(reinterpret_cast<const float4*>(Ph + (int64_t)i * D + c0 + c4))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // row j of the chunk: sequence b = (r0 + j) / R, member g = (r0 + j) % R
+    // (a query head for g < G, else new key g - G); 8 elements per thread and step
+    constexpr int QV = 8;
+    float xv[kRotRows * 128 / 256];
+#pragma unroll
+    for (int u = 0; u < kRotRows * 128 / 256 / QV; ++u) {
+        const int it = (tid + u * 256) * QV;
+        const int j = it / D, i = it % D;
+        const int64_t jr = r0 + j;
+        const Tp* src = nullptr;
+        if (j < nrows) {
+            const int b = (int)(jr / R), g = (int)(jr % R);
+            src = g < G ? q + ((int64_t)b * H_q + (int64_t)hk * G + g) * D
+                        : K_new + (((int64_t)b * H_kv + hk) * T + (g - G)) * D;
+        }
+#pragma unroll
+        for (int e = 0; e < QV; ++e) xv[u * QV + e] = src ? E::load1(src + i + e) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int it = tid + u * 256;
+        const int i = it >> 3, c4 = (it & 7) * 4;
+        if (i < 128) *reinterpret_cast<float4*>(&Ps[i][c4]) = pv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kRotRows * 128 / 256 / QV; ++u) {
+        const int it = (tid + u * 256) * QV;
+        const int j = it / D, i = it % D;
+#pragma unroll
+        for (int e = 0; e < QV; ++e) xs[j][i + e] = xv[u * QV + e];
+    }
+    __syncthreads();
+    for (int j = warp; j < nrows; j += 8) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) acc = fmaf(xs[j][i], Ps[i][lane], acc);
+        const int64_t jr = r0 + j;
+        const int b = (int)(jr / R), g = (int)(jr % R);
+        const int c = c0 + lane;
+        if (g < G) {
+            if (c < D) q_rot[((int64_t)b * H_q + (int64_t)hk * G + g) * D + c] = acc;
+        } else {
+            const int t = g - G;
+            const int64_t row = ((int64_t)b * H_kv + hk) * S_max + pos + t;
+            const Tp kt = E::from_float(acc);
+            if (c < D) Kt_cache[row * D + c] = kt;
+            if (Kt_lo != nullptr && c < d_lo) Kt_lo[row * d_lo + c] = kt;
+            if (cb == 0) {  // one column block copies the value row
+                const Tp* vs = V_new + (((int64_t)b * H_kv + hk) * T + t) * D;
+                for (int e = lane; e < D; e += 32) V_cache[row * D + e] = vs[e];
+            }
+        }
+    }
+    // hold: launched beside the score scan, this grid completes only after the
+    // scan does (one waiting thread is enough), so the kernels that wait on
+    // it also see the scan's scores
+    if (hold && threadIdx.x == 0 && blockIdx.x == 0) griddep_wait();
+}
+
+cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V_new,
+                          const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
+                          int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
+                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl) {
+    const int G = q != nullptr ? H_q / H_kv : 0;
+    const int Tn = K_new != nullptr ? T : 0;
+    const int R = G + Tn;
+    if (R == 0) return cudaSuccess;
+    const int64_t chunks = ((int64_t)B * R + kRotRows - 1) / kRotRows;
+    const int64_t nblocks = chunks * H_kv * ((D + kRotCols - 1) / kRotCols);
+    if (nblocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)nblocks);
+    const int hold = pdl ? 1 : 0;
+    if (dt == kF32)
+        return launch_kernel(k_rotate_rows<ElemF32>, grid, dim3(256), 0, s, pdl,
+                             static_cast<const float*>(q), static_cast<const float*>(K_new),
+                             static_cast<const float*>(V_new), P, q_rot,
+                             static_cast<float*>(Kt_cache), static_cast<float*>(V_cache),
+                             static_cast<float*>(Kt_lo), d_lo, B, H_q, H_kv, G, Tn, D, S_max, pos,
+                             done, n_done, hold);
+    using T16 = __nv_bfloat16;
+    return launch_kernel(k_rotate_rows<ElemBF16>, grid, dim3(256), 0, s, pdl,
+                         static_cast<const T16*>(q), static_cast<const T16*>(K_new),
+                         static_cast<const T16*>(V_new), P, q_rot, static_cast<T16*>(Kt_cache),
+                         static_cast<T16*>(V_cache), static_cast<T16*>(Kt_lo), d_lo, B, H_q, H_kv,
+                         G, Tn, D, S_max, pos, done, n_done, hold);
+}
+
+cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
+                                 int D, float* q_rot, cudaStream_t s, int* done, int n_done,
+                                 bool pdl) {
+    return launch_rotate(dt, q, nullptr, nullptr, P, q_rot, nullptr, nullptr, nullptr, 0, B, H_q,
+                         H_kv, 0, D, 0, 0, s, done, n_done, pdl);
+}
+
+cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
+                          void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
+                          int T, int D, int64_t S_max, int64_t pos, cudaStream_t s) {
+    return launch_rotate(dt, nullptr, K_new, V_new, P, nullptr, Kt_cache, V_cache, Kt_lo, d_lo, B,
+                         H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0, false);
+}
+
+}  // namespace loki

@@ -1,9 +1,8 @@
-// Query rotation and the (register-staged) low-dimensional score scan of Loki.
+// The (register-staged) low-dimensional score scan of Loki.
 //
 // Loki (NeurIPS 2024 poster page, TL;DR and "Visual Insights" Figure 1
-// caption; briefgpt.xyz abstract page): the query is projected onto the PCA
-// basis and every cached token is scored on the first d principal components
-// only, s_j = q~[:d] . K~_j[:d].
+// caption; briefgpt.xyz abstract page): every cached token is scored on the
+// first d principal components only, s_j = q~[:d] . K~_j[:d], with q~ = q P.
 //
 // The scan is an HBM stream over d of the D columns of each cached row. Each
 // row's d columns are covered by L = next_pow2(ceil(d * elem / 16)) lanes,
@@ -15,88 +14,6 @@
 #include "launch.h"
 
 namespace loki {
-
-// q_rot[row, c] = sum_i q[row, i] P[h_kv, i, c]; also zeroes done[0, n_done)
-// (the attention kernel's per-row counters) when done is given. One CTA per (KV head, block of
-// 32 output columns, chunk of up to 32 query rows of that head): the P column
-// block (128 x 32 fp32) is staged once in shared memory and reused by every
-// query of the head; each warp computes one query's 32 columns per step.
-constexpr int kProjCols = 32;
-constexpr int kProjRows = 32;
-
-template <class E>
-__global__ void __launch_bounds__(256) k_project_query(const typename E::T* __restrict__ q,
-                                                       const float* __restrict__ P,
-                                                       float* __restrict__ q_rot, int B, int H_q,
-                                                       int G, int D, int* __restrict__ done,
-                                                       int n_done, int hold) {
-    __shared__ float Ps[128][kProjCols];
-    __shared__ float qs[kProjRows][128];
-    // the next kernel (the score scan) may start streaming keys right away
-    griddep_launch_dependents();
-    if (done != nullptr) {
-        const int nb = gridDim.x * gridDim.y * gridDim.z;
-        const int bid = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-        for (int i = bid * 256 + (int)threadIdx.x; i < n_done; i += nb * 256) done[i] = 0;
-    }
-    const int hk = blockIdx.x;
-    const int c0 = blockIdx.y * kProjCols;
-    const int r0 = blockIdx.z * kProjRows;
-    const int nrows = min(kProjRows, B * G - r0);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float* Ph = P + (int64_t)hk * D * D;
-    // P block: 128 rows x 32 columns = 1024 float4, 4 per thread, all in flight
-    float4 pv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int it = tid + u * 256;
-        const int i = it >> 3, c4 = (it & 7) * 4;
-        pv[u] = (i < D && c0 + c4 < D)
-                    ? __ldg(reinterpret_cast<const float4*>(Ph + (int64_t)i * D + c0 + c4))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // the head's queries: row j of the chunk is (batch b, group member g);
-    // 8 consecutive elements per thread per step
-    constexpr int QV = 8;
-    float qv[kProjRows * 128 / 256];
-#pragma unroll
-    for (int u = 0; u < kProjRows * 128 / 256 / QV; ++u) {
-        const int it = (tid + u * 256) * QV;
-        const int j = it / D, i = it % D;
-        const int jr = r0 + j;
-        const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
-#pragma unroll
-        for (int e = 0; e < QV; ++e)
-            qv[u * QV + e] = (j < nrows) ? E::load1(q + row * D + i + e) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int it = tid + u * 256;
-        const int i = it >> 3, c4 = (it & 7) * 4;
-        if (i < 128) *reinterpret_cast<float4*>(&Ps[i][c4]) = pv[u];
-    }
-#pragma unroll
-    for (int u = 0; u < kProjRows * 128 / 256 / QV; ++u) {
-        const int it = (tid + u * 256) * QV;
-        const int j = it / D, i = it % D;
-#pragma unroll
-        for (int e = 0; e < QV; ++e) qs[j][i + e] = qv[u * QV + e];
-    }
-    __syncthreads();
-    for (int j = warp; j < nrows; j += 8) {
-        float acc = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; ++i) acc = fmaf(qs[j][i], Ps[i][lane], acc);
-        const int jr = r0 + j;
-        const int64_t row = (int64_t)(jr / G) * H_q + (int64_t)hk * G + jr % G;
-        if (c0 + lane < D) q_rot[row * D + c0 + lane] = acc;
-    }
-    // hold: launched beside the score scan, this grid completes only after the
-    // scan does (one waiting thread is enough), so the kernels that wait on
-    // it also see the scan's scores
-    if (hold && threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-        griddep_wait();
-}
 
 template <class E, int G>
 __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ q_rot,
@@ -171,21 +88,6 @@ __global__ void __launch_bounds__(256) k_score_lowdim(const float* __restrict__ 
         }
         r += seg;
     }
-}
-
-cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
-                                 int D, float* q_rot, cudaStream_t s, int* done, int n_done,
-                                 bool pdl) {
-    const int G = H_q / H_kv;
-    dim3 grid(H_kv, (D + kProjCols - 1) / kProjCols, (B * G + kProjRows - 1) / kProjRows);
-    const int hold = pdl ? 1 : 0;
-    if (dt == kF32)
-        return launch_kernel(k_project_query<ElemF32>, grid, dim3(256), 0, s, pdl,
-                             static_cast<const float*>(q), P, q_rot, B, H_q, G, D, done, n_done,
-                             hold);
-    return launch_kernel(k_project_query<ElemBF16>, grid, dim3(256), 0, s, pdl,
-                         static_cast<const __nv_bfloat16*>(q), P, q_rot, B, H_q, G, D, done,
-                         n_done, hold);
 }
 
 template <class E, int G>

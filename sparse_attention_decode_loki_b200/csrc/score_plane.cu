@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
     const float* __restrict__ P, const typename E::T* __restrict__ Klo,
     float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
-    int D, int d, int64_t total, int64_t per) {
+    int D, int d, int64_t total, int64_t per, int wait_row) {
     constexpr int KV = E::kVec;
     constexpr int kRowBytes = NV * 16;
     constexpr int kTR = kScoreConsumers;  // rows per tile
@@ -92,6 +92,9 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
             const uint64_t pol = l2_policy_evict_first();
             int i = 0;
             bool ok = true;
+            // rows [wait_row, S) of every unit are written by the preceding
+            // kernel (an append): wait for it before the first tile holding one
+            bool waited = wait_row >= S;
             for (int64_t r = R0; r < R1 && ok;) {
                 const int64_t unit = r / S;
                 const int s0 = (int)(r - unit * S);
@@ -105,12 +108,20 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
                         ok = false;
                         break;
                     }
+                    if (!waited && s0 + t0 + n > wait_row) {
+                        griddep_wait();
+                        fence_proxy_async_global();  // its stores, then our bulk reads
+                        waited = true;
+                    }
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(n * kRowBytes));
                     bulk_load_hint(ring + (size_t)st * kTile, src + (int64_t)t0 * kRowBytes,
                                    (uint32_t)(n * kRowBytes), &full[st], pol);
                 }
                 r += seg;
             }
+            // a CTA that never met a new row still completes only after the
+            // preceding kernel, so the kernels after the scan see its writes
+            if (!waited) griddep_wait();
             // every issued copy has landed before the CTA may exit
             for (int j = max(0, i - kStages); j < i; ++j)
                 mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, err);
@@ -244,6 +255,7 @@ struct PlaneArgs {
     int B, H_q, H_kv;
     int64_t S, S_max;
     int D, d;
+    int64_t wait_row;  // first row written by the preceding kernel (>= S: none)
 };
 
 template <class E, int G, int NV, bool kFuseQ>
@@ -271,7 +283,8 @@ static cudaError_t plane_impl(const PlaneArgs& a, cudaStream_t s, bool pdl) {
     using T = typename E::T;
     return launch_kernel(kern, dim3((unsigned)grid), dim3(kScoreThreads), smem, s, pdl, a.q_rot,
                          static_cast<const T*>(a.q), a.P, static_cast<const T*>(a.Klo), a.scores,
-                         a.err, a.H_q, a.H_kv, (int)a.S, a.S_max, a.D, a.d, total, per);
+                         a.err, a.H_q, a.H_kv, (int)a.S, a.S_max, a.D, a.d, total, per,
+                         (int)(a.wait_row < a.S ? a.wait_row : a.S));
 }
 
 template <class E, int G, int NV>
@@ -323,7 +336,7 @@ bool score_plane_fuses(Dt dt, int G, int d_lo, int D) {
 cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B, int H_q,
                                int H_kv, int64_t S, int64_t S_max, int D, int d_lo, int d,
                                float* scores, cudaStream_t s, bool pdl, const void* q,
-                               const float* P) {
+                               const float* P, int64_t wait_row) {
     int* err = device_error_word();
     if (err == nullptr) return cudaErrorInvalidDevice;
     const int G = H_q / H_kv;
@@ -336,11 +349,12 @@ cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B
     const int nv = d_lo * (dt == kF32 ? 4 : 2) / 16;
     const bool fuse = q != nullptr && P != nullptr;
     if (fuse && D != 128) return cudaErrorInvalidValue;  // the fused rotation takes head dim 128
-    // a scan that rotates its own queries reads q at once: it is ordered
-    // normally after the preceding work, never launched early beside it
-    if (fuse) pdl = false;
+    // a scan that rotates its own queries reads q and P at once: it is
+    // launched early beside the preceding kernel only when that kernel writes
+    // cache rows the producer waits for (an append), never q or P
+    if (fuse && wait_row >= S) pdl = false;
     const PlaneArgs a{q_rot, fuse ? q : nullptr, fuse ? P : nullptr, Klo, scores, err, B, H_q,
-                      H_kv, S, S_max, D, d};
+                      H_kv, S, S_max, D, d, wait_row};
     if (dt == kF32) return plane_dispatch<ElemF32>(G, nv, a, s, pdl);
     return plane_dispatch<ElemBF16>(G, nv, a, s, pdl);
 }

@@ -107,6 +107,12 @@ __device__ __forceinline__ void bulk_load_hint(void* dst_smem, const void* src, 
         : "memory");
 }
 
+// order this thread's earlier generic-proxy view of global memory before its
+// later asynchronous-proxy (bulk copy) accesses
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // named barrier over `count` threads (a multiple of 32), id 1..15
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
