@@ -70,9 +70,9 @@ LOKI_API const char* loki_status_string(loki_status st);
 LOKI_API const char* loki_last_error(void);
 
 /*
- * Kernel error word of the current device: nonzero (1) if a staged kernel's
- * bounded wait on an asynchronous copy gave up (its results are then
- * invalid). Synchronous: copies 4 bytes from the device (waiting for prior
+ * Kernel error word of the current device: 1 if a staged kernel's bounded
+ * wait on an asynchronous copy gave up, 2 if a paged call met a block-table
+ * entry outside the page pool (the results of the call are then invalid). Synchronous: copies 4 bytes from the device (waiting for prior
  * work); with reset != 0 the word is cleared afterwards.
  */
 LOKI_API loki_status loki_device_error(int* code, int reset);
@@ -231,6 +231,68 @@ LOKI_API loki_status loki_decode_attention_noalloc(const void* q, const void* Kt
                                                    int D, int d, int64_t k, float scale,
                                                    loki_dtype dt, void* out, int32_t* selected_idx,
                                                    void* stream);
+
+/* Ragged batches over a paged KV-cache ------------------------------------- */
+/*
+ * The Loki pages evaluate one prompt length at a time and say nothing about
+ * batches of sequences with their own lengths or about cache memory layout;
+ * these entry points carry the same decode step (and append) to the paged
+ * layout of serving engines. Every sequence b keeps its own length S_b, and
+ * the selection keeps min(k, S_b) tokens (the plainest reading when a
+ * sequence holds fewer than k).
+ *
+ * Page pool layout (all dt, 16-byte aligned, caller-owned):
+ *   Kt_pages, V_pages  [n_pages, H_kv, page_size, D]    rotated keys, values
+ *   Kt_lo_pages        [n_pages, H_kv, page_size, d_lo] low-dimensional key plane
+ *   block_table        [B, max_pages] int32: sequence b's token j lives in page
+ *                      block_table[b][j / page_size], row j % page_size
+ * A contiguous cache [B, H_kv, S_max, D] is the case page_size = S_max,
+ * max_pages = 1, block_table[b][0] = b. Limits: page_size * max_pages <=
+ * 262144 tokens per sequence; n_pages * H_kv * page_size < 2^31 rows. Page
+ * numbers outside [0, n_pages) are not followed: the token is skipped (the
+ * decode) or not written (the append), and loki_device_error then reports 2.
+ */
+
+/* Bytes of workspace loki_decode_attention_paged needs. */
+LOKI_API size_t loki_paged_decode_workspace_size(int B, int H_q, int H_kv, int page_size,
+                                                 int max_pages, int D, int d, int64_t k);
+
+/*
+ * One decode step per sequence over its own S_b = seq_lens[b] cached tokens
+ * (device array, int32; values are clamped to [0, page_size * max_pages]; a
+ * sequence with S_b = 0 gives zeros and no selection). Otherwise as
+ * loki_decode_attention_plane: same selection rule and arithmetic, over the
+ * token indices j < S_b of each sequence.
+ *   out          [B, H_q, D] (dt)
+ *   selected_idx [B, H_q, k] int32: the min(k, S_b) selected token indices
+ *                ascending, then -1
+ * The scan reads the plane pages (d <= d_lo; plane rows of 16, 32, 64 or 128
+ * bytes with (H_q / H_kv) * d_lo <= 64 elements), the attention the key and
+ * value pages.
+ */
+LOKI_API loki_status loki_decode_attention_paged(const void* q, const void* Kt_pages,
+                                                 const void* V_pages, const void* Kt_lo_pages,
+                                                 int d_lo, const float* P,
+                                                 const int32_t* block_table,
+                                                 const int32_t* seq_lens, int B, int H_q, int H_kv,
+                                                 int page_size, int max_pages, int64_t n_pages,
+                                                 int D, int d, int64_t k, float scale,
+                                                 loki_dtype dt, void* out, int32_t* selected_idx,
+                                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * loki_append_keys into the page pool: the T new tokens of sequence b become
+ * its tokens positions[b] + t (positions: device array, int32), their rotated
+ * keys (and plane rows when Kt_lo_pages is not NULL) and values written into
+ * the pages block_table names. Same arithmetic as loki_append_keys.
+ *   K_new, V_new [B, H_kv, T, D] (dt)
+ */
+LOKI_API loki_status loki_append_keys_paged(const void* K_new, const void* V_new, const float* P,
+                                            void* Kt_pages, void* V_pages, void* Kt_lo_pages,
+                                            int d_lo, const int32_t* block_table,
+                                            const int32_t* positions, int B, int H_kv, int T,
+                                            int page_size, int max_pages, int64_t n_pages, int D,
+                                            loki_dtype dt, void* stream);
 
 /* Steps of loki_decode_attention, callable one by one ------------------- */
 

@@ -23,7 +23,8 @@ __all__ = [
     "LokiError", "LIB_PATH",
     "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
     "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_fused",
-    "loki_decode_step",
+    "loki_decode_step", "loki_decode_attention_paged", "loki_append_keys_paged",
+    "loki_paged_decode_workspace_size",
     "loki_decode_attention_noalloc",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
@@ -270,6 +271,86 @@ def loki_decode_step(q: torch.Tensor, K_new: torch.Tensor, V_new: torch.Tensor, 
                                selected_idx.data_ptr(), ws.data_ptr(), _ws_bytes(ws),
                                _stream(dev)), "loki_decode_step")
     return out, selected_idx
+
+
+def loki_paged_decode_workspace_size(B: int, H_q: int, H_kv: int, page_size: int,
+                                     max_pages: int, D: int, d: int, k: int) -> int:
+    return int(lib.loki_paged_decode_workspace_size(B, H_q, H_kv, page_size, max_pages, D, d, k))
+
+
+def _check_pages(Kt_pages, V_pages, Kt_lo_pages, block_table):
+    if Kt_pages.dim() != 4 or V_pages.shape != Kt_pages.shape:
+        raise ValueError("Kt_pages and V_pages must be [n_pages, H_kv, page_size, D]")
+    if Kt_lo_pages is not None and (Kt_lo_pages.dim() != 4 or
+                                    Kt_lo_pages.shape[:3] != Kt_pages.shape[:3] or
+                                    Kt_lo_pages.dtype != Kt_pages.dtype):
+        raise ValueError("Kt_lo_pages must be [n_pages, H_kv, page_size, d_lo] with the pages' dtype")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise TypeError("block_table must be int32 [B, max_pages]")
+    return Kt_pages.shape
+
+
+def loki_decode_attention_paged(q: torch.Tensor, Kt_pages: torch.Tensor, V_pages: torch.Tensor,
+                                Kt_lo_pages: torch.Tensor, P: torch.Tensor,
+                                block_table: torch.Tensor, seq_lens: torch.Tensor, d: int, k: int,
+                                scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                selected_idx: Optional[torch.Tensor] = None,
+                                workspace: Optional[torch.Tensor] = None
+                                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode a ragged batch over a paged cache (see include/loki.h).
+    Returns (out [B, H_q, D], selected_idx [B, H_q, k] int32, -1 padded)."""
+    dev = _cuda(q, Kt_pages, V_pages, Kt_lo_pages, P, block_table, seq_lens)
+    n_pages, H_kv, page_size, D = _check_pages(Kt_pages, V_pages, Kt_lo_pages, block_table)
+    B, H_q, Dq = q.shape
+    if Dq != D or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("q [B, H_q, D], block_table [B, max_pages], seq_lens [B] disagree")
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    if Kt_pages.dtype != q.dtype or V_pages.dtype != q.dtype:
+        raise TypeError("q and the pages must share a dtype")
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if selected_idx is None:
+        selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    _cuda(q, out, selected_idx)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    ws = _ws(loki_paged_decode_workspace_size(B, H_q, H_kv, page_size, max_pages, D, d, k), dev,
+             workspace)
+    check(lib.loki_decode_attention_paged(q.data_ptr(), Kt_pages.data_ptr(), V_pages.data_ptr(),
+                                          Kt_lo_pages.data_ptr(), Kt_lo_pages.shape[3],
+                                          P.data_ptr(), block_table.data_ptr(),
+                                          seq_lens.data_ptr(), B, H_q, H_kv, page_size, max_pages,
+                                          n_pages, D, d, k, float(scale), _dt(q), out.data_ptr(),
+                                          selected_idx.data_ptr(), ws.data_ptr(), _ws_bytes(ws),
+                                          _stream(dev)), "loki_decode_attention_paged")
+    return out, selected_idx
+
+
+def loki_append_keys_paged(K_new: torch.Tensor, V_new: torch.Tensor, P: torch.Tensor,
+                           Kt_pages: torch.Tensor, V_pages: torch.Tensor,
+                           block_table: torch.Tensor, positions: torch.Tensor,
+                           Kt_lo_pages: Optional[torch.Tensor] = None) -> None:
+    """Rotate K_new [B, H_kv, T, D] by P into the page pool at tokens positions[b] + t."""
+    dev = _cuda(K_new, V_new, P, Kt_pages, V_pages, block_table, positions,
+                *(() if Kt_lo_pages is None else (Kt_lo_pages,)))
+    n_pages, H_kv, page_size, D = _check_pages(Kt_pages, V_pages, Kt_lo_pages, block_table)
+    B, Hk, T, Dk = K_new.shape
+    if Hk != H_kv or Dk != D or V_new.shape != K_new.shape or tuple(positions.shape) != (B,):
+        raise ValueError("K_new, V_new [B, H_kv, T, D] and positions [B] must match the pages")
+    if positions.dtype != torch.int32:
+        raise TypeError("positions must be int32")
+    for t in (V_new, Kt_pages, V_pages):
+        if t.dtype != K_new.dtype:
+            raise TypeError("K_new, V_new and the pages must share a dtype")
+    check(lib.loki_append_keys_paged(K_new.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+                                     Kt_pages.data_ptr(), V_pages.data_ptr(),
+                                     Kt_lo_pages.data_ptr() if Kt_lo_pages is not None else None,
+                                     Kt_lo_pages.shape[3] if Kt_lo_pages is not None else 0,
+                                     block_table.data_ptr(), positions.data_ptr(), B, H_kv, T,
+                                     page_size, block_table.shape[1], n_pages, D, _dt(K_new),
+                                     _stream(dev)), "loki_append_keys_paged")
 
 
 def loki_decode_attention_fused(q: torch.Tensor, Kt_cache: torch.Tensor, V_cache: torch.Tensor,

@@ -53,6 +53,16 @@ PROTOTYPES = {
     "loki_decode_attention_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                               c_int, c_int64, c_int64, c_int, c_int, c_int64,
                                               c_float, c_int, c_void_p, c_void_p, c_void_p]),
+    "loki_paged_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int,
+                                                    c_int, c_int64]),
+    "loki_decode_attention_paged": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                            c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                            c_int, c_int, c_int64, c_int, c_int, c_int64, c_float,
+                                            c_int, c_void_p, c_void_p, c_void_p, c_size_t,
+                                            c_void_p]),
+    "loki_append_keys_paged": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_int, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
+                                       c_int, c_int64, c_int, c_int, c_void_p]),
     "loki_project_query": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p,
                                    c_void_p]),
     "loki_score_lowdim": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int64, c_int64, c_int,

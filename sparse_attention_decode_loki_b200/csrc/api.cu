@@ -119,6 +119,20 @@ DecodeWs decode_ws(int B, int H_q, int64_t S, int D, int64_t k) {
     return w;
 }
 
+// Paged decode: the work-split area of the paged scan, then a decode
+// workspace for rows of S_cap = page_size * max_pages scores.
+constexpr int kPagedMaxGrid = 1024;  // >= the scan grid (one CTA per SM)
+struct PagedWs {
+    size_t start, dec, total;
+};
+PagedWs paged_ws(int B, int H_q, int64_t S_cap, int D, int64_t k) {
+    PagedWs w;
+    w.start = 0;
+    w.dec = align_up(loki::paged_start_bytes(B, kPagedMaxGrid));
+    w.total = w.dec + decode_ws(B, H_q, S_cap, D, k).total;
+    return w;
+}
+
 struct SparseWs {
     size_t done, ml, acc, total;
 };
@@ -457,6 +471,129 @@ loki_status loki_decode_step(const void* q, const void* K_new, const void* V_new
     return decode_impl("loki_decode_step", q, Kt_cache, V_cache, Kt_lo, d_lo, P, B, H_q, H_kv,
                        pos + T, S_max, D, d, k, scale, dt, out, selected_idx, ws, ws_bytes, stream,
                        K_new, V_new, T);
+}
+
+static loki_status check_pages(int page_size, int max_pages, int64_t n_pages, int H_kv) {
+    LOKI_REQUIRE(page_size >= 1 && max_pages >= 1 && n_pages >= 1, LOKI_ERR_INVALID_ARG,
+                 "page_size, max_pages and n_pages must be >= 1");
+    LOKI_REQUIRE((int64_t)page_size * max_pages <= kMaxS, LOKI_ERR_UNSUPPORTED,
+                 "page_size * max_pages must be < 2^31 tokens");
+    LOKI_REQUIRE(n_pages * H_kv * (int64_t)page_size <= kMaxS, LOKI_ERR_UNSUPPORTED,
+                 "the page pool must hold fewer than 2^31 rows (n_pages * H_kv * page_size)");
+    return LOKI_OK;
+}
+
+size_t loki_paged_decode_workspace_size(int B, int H_q, int H_kv, int page_size, int max_pages,
+                                        int D, int d, int64_t k) {
+    (void)H_kv;
+    (void)d;
+    if (B < 1 || H_q < 1 || page_size < 1 || max_pages < 1 || D < 1 || k < 1) return 0;
+    return paged_ws(B, H_q, (int64_t)page_size * max_pages, D, k).total;
+}
+
+loki_status loki_decode_attention_paged(const void* q, const void* Kt_pages, const void* V_pages,
+                                        const void* Kt_lo_pages, int d_lo, const float* P,
+                                        const int32_t* block_table, const int32_t* seq_lens,
+                                        int B, int H_q, int H_kv, int page_size, int max_pages,
+                                        int64_t n_pages, int D, int d, int64_t k, float scale,
+                                        loki_dtype dt, void* out, int32_t* selected_idx,
+                                        void* ws, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_q, H_kv, D));
+    LOKI_CHECK(check_pages(page_size, max_pages, n_pages, H_kv));
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    const int64_t S_cap = (int64_t)page_size * max_pages;
+    LOKI_REQUIRE(d >= 1 && d <= d_lo, LOKI_ERR_INVALID_ARG, "d must be in [1, d_lo] (got %d)", d);
+    LOKI_REQUIRE(k >= 1 && k <= S_cap, LOKI_ERR_INVALID_ARG,
+                 "k must be in [1, page_size * max_pages] (got %lld)", (long long)k);
+    const loki::Dt t = to_dt(dt);
+    LOKI_REQUIRE(loki::paged_scan_supported(t, H_q / H_kv, d_lo), LOKI_ERR_UNSUPPORTED,
+                 "the paged scan takes plane rows of 16, 32, 64 or 128 bytes with "
+                 "(H_q / H_kv) * d_lo <= 64 elements");
+    LOKI_REQUIRE(S_cap <= 262144, LOKI_ERR_UNSUPPORTED,
+                 "paged decode selects from at most 262144 tokens per sequence");
+    LOKI_PTR(q, 16);
+    LOKI_PTR(Kt_pages, 16);
+    LOKI_PTR(V_pages, 16);
+    LOKI_PTR(Kt_lo_pages, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(block_table, 4);
+    LOKI_PTR(seq_lens, 4);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_PTR(ws, 256);
+    const PagedWs pw = paged_ws(B, H_q, S_cap, D, k);
+    LOKI_REQUIRE(ws_bytes >= pw.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, pw.total);
+    const int grid = loki::paged_scan_grid();
+    LOKI_REQUIRE(grid >= 1 && grid <= kPagedMaxGrid, LOKI_ERR_CUDA, "no usable current CUDA device");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const char* name = "loki_decode_attention_paged";
+    void* start_ws = at<char>(ws, pw.start);
+    void* dws = at<char>(ws, pw.dec);
+    const DecodeWs w = decode_ws(B, H_q, S_cap, D, k);
+    float* q_rot = at<float>(dws, w.q_rot);
+    float* scores = at<float>(dws, w.scores);
+    int* done = at<int>(dws, w.done);
+    const int rows = B * H_q;
+    // the rotated queries (and zeroed row counters), the lengths' work split,
+    // the paged scan, then top-k per row length and the paged gather
+    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows), name);
+    LOKI_CUDA(loki::launch_paged_prefix(seq_lens, B, H_kv, S_cap, start_ws, grid, s), name);
+    LOKI_CUDA(loki::launch_score_paged(t, q_rot, Kt_lo_pages, d_lo, block_table, start_ws, B, H_q,
+                                       H_kv, page_size, max_pages, n_pages, S_cap, d, scores, grid,
+                                       s),
+              name);
+    const int* lens = loki::paged_lens(start_ws, B);
+    LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S_cap, k, selected_idx, s, true, lens, H_q),
+              name);
+    loki::PagedKV pg;
+    pg.block_table = block_table;
+    pg.page_size = page_size;
+    pg.max_pages = max_pages;
+    pg.n_pages = n_pages;
+    pg.lens = lens;
+    LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_pages, V_pages, selected_idx, B, H_q, H_kv,
+                                            S_cap, S_cap, D, k, resolve_scale(scale, D), out,
+                                            at<float2>(dws, w.ml), at<float>(dws, w.acc), done, s,
+                                            true, pg),
+              name);
+    return LOKI_OK;
+}
+
+loki_status loki_append_keys_paged(const void* K_new, const void* V_new, const float* P,
+                                   void* Kt_pages, void* V_pages, void* Kt_lo_pages, int d_lo,
+                                   const int32_t* block_table, const int32_t* positions, int B,
+                                   int H_kv, int T, int page_size, int max_pages, int64_t n_pages,
+                                   int D, loki_dtype dt, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_kv, H_kv, D));
+    LOKI_CHECK(check_pages(page_size, max_pages, n_pages, H_kv));
+    LOKI_REQUIRE(T >= 1, LOKI_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    LOKI_PTR(K_new, 16);
+    LOKI_PTR(V_new, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(Kt_pages, 16);
+    LOKI_PTR(V_pages, 16);
+    LOKI_PTR(block_table, 4);
+    LOKI_PTR(positions, 4);
+    if (Kt_lo_pages != nullptr) {
+        LOKI_CHECK(check_plane(d_lo, D, dt));
+        LOKI_PTR(Kt_lo_pages, 16);
+    }
+    loki::PagedKV pg;
+    pg.block_table = block_table;
+    pg.page_size = page_size;
+    pg.max_pages = max_pages;
+    pg.n_pages = n_pages;
+    LOKI_CUDA(loki::launch_rotate(to_dt(dt), nullptr, K_new, V_new, P, nullptr, Kt_pages, V_pages,
+                                  Kt_lo_pages, Kt_lo_pages != nullptr ? d_lo : 0, B, H_kv, H_kv, T,
+                                  D, 0, 0, static_cast<cudaStream_t>(stream), nullptr, 0, false,
+                                  &pg, positions),
+              "loki_append_keys_paged");
+    return LOKI_OK;
 }
 
 loki_status loki_decode_attention_fused(const void* q, const void* Kt_cache, const void* V_cache,

@@ -58,8 +58,10 @@ cudaError_t launch_score_plane(Dt dt, const float* q_rot, const void* Klo, int B
                                float* scores, cudaStream_t s, bool pdl, const void* q = nullptr,
                                const float* P = nullptr, int64_t wait_row = INT64_MAX);
 
+// With lens, row r holds min(lens[r / H_q], S) valid keys (at stride S) and
+// selects min(k, that) of them, padding its k outputs with -1.
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
-                        cudaStream_t s, bool pdl);
+                        cudaStream_t s, bool pdl, const int* lens = nullptr, int H_q = 1);
 
 // Whether the fused one-CTA-per-unit decode kernel can run this decode over a
 // low-dim key plane: head dim 128; G in {1, 2, 4, 8}; S within the block
@@ -91,11 +93,37 @@ cudaError_t launch_select_attend(Dt dt, const float* scores, const float* q_rot,
 int64_t sparse_max_parts(int64_t rows, int64_t k);
 // done[B*H_q] must be zero on entry (per-row completion counters; the last
 // warp of a row merges its partials into out and leaves the counter at zero).
+// Paged caches (block_table not null): Kt and V are page pools [n_pages, H_kv,
+// page_size, D]; sequence b's token j is row j % page_size of page
+// block_table[b * max_pages + j / page_size]. With lens, tokens at or beyond
+// lens[b] (and pages outside the pool) are skipped.
+struct PagedKV {
+    const int* block_table = nullptr;
+    int page_size = 0;
+    int max_pages = 0;
+    int64_t n_pages = 0;
+    const int* lens = nullptr;
+};
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
                                     float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                                    bool pdl);
+                                    bool pdl, const PagedKV& pg = PagedKV());
+
+// ---- paged key plane -------------------------------------------------------
+// One CTA per SM; the prefix kernel turns seq_lens into this grid's work split.
+int paged_scan_grid();
+// Bytes of the work-split area (lengths, row offsets, per-CTA starts).
+size_t paged_start_bytes(int B, int grid);
+bool paged_scan_supported(Dt dt, int G, int d_lo);
+cudaError_t launch_paged_prefix(const int* seq_lens, int B, int H_kv, int64_t S_cap, void* start_ws,
+                                int grid, cudaStream_t s);
+// the clamped per-sequence lengths inside the work-split area
+const int* paged_lens(const void* start_ws, int B);
+cudaError_t launch_score_paged(Dt dt, const float* q_rot, const void* Klo_pages, int d_lo,
+                               const int* block_table, const void* start_ws, int B, int H_q,
+                               int H_kv, int page_size, int max_pages, int64_t n_pages,
+                               int64_t S_cap, int d, float* scores, int grid, cudaStream_t s);
 
 // split-S partial slots per (batch, KV head) unit
 int64_t dense_max_parts(int64_t S);
@@ -109,10 +137,14 @@ cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int
 // Kt_lo when not null) with their values copied to V_cache (K_new may be
 // null). Also zeroes done[0, n_done). With pdl it is a programmatic dependent
 // of the preceding kernel that completes only after it (see the score scan).
+// Paged (pg not null): the new keys of sequence b go to logical tokens
+// positions[b] + t of its pages (rows whose page is missing are skipped and
+// flag the device error word).
 cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V_new,
                           const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
                           int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
-                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl);
+                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl,
+                          const PagedKV* pg = nullptr, const int* positions = nullptr);
 
 // ---- supporting subsystems -----------------------------------------------
 // Kt_lo (may be null): [B, H_kv, S_max, d_lo] plane that also receives the

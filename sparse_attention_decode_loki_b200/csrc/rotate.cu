@@ -27,7 +27,9 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
     const typename E::T* __restrict__ V_new, const float* __restrict__ P, float* __restrict__ q_rot,
     typename E::T* __restrict__ Kt_cache, typename E::T* __restrict__ V_cache,
     typename E::T* __restrict__ Kt_lo, int d_lo, int B, int H_q, int H_kv, int G, int T, int D,
-    int64_t S_max, int64_t pos, int* __restrict__ done, int n_done, int hold) {
+    int64_t S_max, int64_t pos, int* __restrict__ done, int n_done, int hold,
+    const int* __restrict__ block_table, const int* __restrict__ positions, int page_size,
+    int max_pages, int64_t n_pages, int* __restrict__ err) {
     using Tp = typename E::T;
     __shared__ float Ps[128][kRotCols];
     __shared__ float xs[kRotRows][128];
@@ -101,7 +103,21 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
             if (c < D) q_rot[((int64_t)b * H_q + (int64_t)hk * G + g) * D + c] = acc;
         } else {
             const int t = g - G;
-            const int64_t row = ((int64_t)b * H_kv + hk) * S_max + pos + t;
+            int64_t row;
+            if (block_table == nullptr) {
+                row = ((int64_t)b * H_kv + hk) * S_max + pos + t;
+            } else {
+                // paged: logical token positions[b] + t of sequence b
+                const int64_t j = (int64_t)positions[b] + t;
+                const int page = (j >= 0 && j < (int64_t)page_size * max_pages)
+                                     ? __ldg(block_table + (int64_t)b * max_pages + j / page_size)
+                                     : -1;
+                if (page < 0 || page >= n_pages) {
+                    if (lane == 0) atomicExch(err, 2);  // nowhere valid to write: skip the row
+                    continue;
+                }
+                row = ((int64_t)page * H_kv + hk) * page_size + j % page_size;
+            }
             const Tp kt = E::from_float(acc);
             if (c < D) Kt_cache[row * D + c] = kt;
             if (Kt_lo != nullptr && c < d_lo) Kt_lo[row * d_lo + c] = kt;
@@ -120,7 +136,14 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
 cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V_new,
                           const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
                           int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
-                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl) {
+                          int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl,
+                          const PagedKV* pg, const int* positions) {
+    int* err = device_error_word();
+    if (err == nullptr) return cudaErrorInvalidDevice;
+    const int* bt = pg != nullptr ? pg->block_table : nullptr;
+    const int ps = pg != nullptr ? pg->page_size : 0;
+    const int mp = pg != nullptr ? pg->max_pages : 0;
+    const int64_t np = pg != nullptr ? pg->n_pages : 0;
     const int G = q != nullptr ? H_q / H_kv : 0;
     const int Tn = K_new != nullptr ? T : 0;
     const int R = G + Tn;
@@ -136,27 +159,27 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
                              static_cast<const float*>(V_new), P, q_rot,
                              static_cast<float*>(Kt_cache), static_cast<float*>(V_cache),
                              static_cast<float*>(Kt_lo), d_lo, B, H_q, H_kv, G, Tn, D, S_max, pos,
-                             done, n_done, hold);
+                             done, n_done, hold, bt, positions, ps, mp, np, err);
     using T16 = __nv_bfloat16;
     return launch_kernel(k_rotate_rows<ElemBF16>, grid, dim3(256), 0, s, pdl,
                          static_cast<const T16*>(q), static_cast<const T16*>(K_new),
                          static_cast<const T16*>(V_new), P, q_rot, static_cast<T16*>(Kt_cache),
                          static_cast<T16*>(V_cache), static_cast<T16*>(Kt_lo), d_lo, B, H_q, H_kv,
-                         G, Tn, D, S_max, pos, done, n_done, hold);
+                         G, Tn, D, S_max, pos, done, n_done, hold, bt, positions, ps, mp, np, err);
 }
 
 cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, int H_q, int H_kv,
                                  int D, float* q_rot, cudaStream_t s, int* done, int n_done,
                                  bool pdl) {
     return launch_rotate(dt, q, nullptr, nullptr, P, q_rot, nullptr, nullptr, nullptr, 0, B, H_q,
-                         H_kv, 0, D, 0, 0, s, done, n_done, pdl);
+                         H_kv, 0, D, 0, 0, s, done, n_done, pdl, nullptr, nullptr);
 }
 
 cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
                           void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
                           int T, int D, int64_t S_max, int64_t pos, cudaStream_t s) {
     return launch_rotate(dt, nullptr, K_new, V_new, P, nullptr, Kt_cache, V_cache, Kt_lo, d_lo, B,
-                         H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0, false);
+                         H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0, false, nullptr, nullptr);
 }
 
 }  // namespace loki

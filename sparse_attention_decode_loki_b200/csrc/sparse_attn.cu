@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int nblk, int64_t N, int64_t W,
     float2* __restrict__ part_ml, float* __restrict__ part_acc, int* __restrict__ done,
-    typename E::T* __restrict__ out) {
+    typename E::T* __restrict__ out, const int* __restrict__ block_table, int page_size,
+    int max_pages, int64_t n_pages, const int* __restrict__ lens, int* __restrict__ err) {
     constexpr int D = 128;
     constexpr int KV = E::kVec;
     constexpr int LPR = D / KV;     // lanes per row
@@ -153,9 +154,13 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
 #pragma unroll
             for (int e = 0; e < KV; ++e) qv[e] = __ldg(qp + e) * scale_log2;
         }
-        const char* Kb = reinterpret_cast<const char*>(Kt) + unit * S_max * kRowBytes + sub * 16;
-        const char* Vb = reinterpret_cast<const char*>(V) + unit * S_max * kRowBytes + sub * 16;
+        // contiguous cache: rows of the unit; paged: rows of the page pool
+        const int64_t base_row = block_table != nullptr ? 0 : unit * S_max;
+        const char* Kb = reinterpret_cast<const char*>(Kt) + base_row * kRowBytes + sub * 16;
+        const char* Vb = reinterpret_cast<const char*>(V) + base_row * kRowBytes + sub * 16;
         const int32_t* ip = idx + r * k;
+        const int S_row = lens != nullptr ? min(S, max(0, lens[b])) : S;
+        const int hk = h / G;
 
         float m = -INFINITY, l = 0.f, acc[KV];
 #pragma unroll
@@ -175,7 +180,18 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
 #pragma unroll
                 for (int u = 0; u < kWarpIdx / 32; ++u) {
                     const int t = lane + 32 * u;
-                    if (t < n) widx[t] = ((unsigned)tk[u] < (unsigned)S) ? tk[u] : -1;
+                    int tok = (t < n && (unsigned)tk[u] < (unsigned)S_row) ? tk[u] : -1;
+                    if (block_table != nullptr && tok >= 0) {
+                        // token -> row of the page pool (< 2^31 rows, checked on the host)
+                        const int page = __ldg(block_table + (int64_t)b * max_pages + tok / page_size);
+                        if (page < 0 || page >= n_pages) {
+                            atomicExch(err, 2);  // a bad block-table entry: skip the token
+                            tok = -1;
+                        } else {
+                            tok = (int)(((int64_t)page * H_kv + hk) * page_size + tok % page_size);
+                        }
+                    }
+                    if (t < n) widx[t] = tok;
                 }
             }
             __syncwarp();
@@ -290,7 +306,7 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
                                const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                int64_t S_max, int D, int64_t k, float scale, void* out,
                                float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                               bool pdl) {
+                               bool pdl, const PagedKV& pg) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
@@ -316,19 +332,20 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     return launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, q_rot,
                          static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv,
                          (int)S, S_max, (int)k, scale * kLog2e, (int)nblk, N, W, part_ml,
-                         part_acc, done, static_cast<T*>(out));
+                         part_acc, done, static_cast<T*>(out), pg.block_table, pg.page_size,
+                         pg.max_pages, pg.n_pages, pg.lens, device_error_word());
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
                                     float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                                    bool pdl) {
+                                    bool pdl, const PagedKV& pg) {
     if (dt == kF32)
         return sparse_impl<ElemF32>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                    part_ml, part_acc, done, s, pdl);
+                                    part_ml, part_acc, done, s, pdl, pg);
     return sparse_impl<ElemBF16>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                 part_ml, part_acc, done, s, pdl);
+                                 part_ml, part_acc, done, s, pdl, pg);
 }
 
 }  // namespace loki

@@ -14,6 +14,7 @@ namespace loki {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kDevErrWaitTimeout = 1;
+constexpr int kDevErrBadPage = 2;  // a block-table entry outside the page pool
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

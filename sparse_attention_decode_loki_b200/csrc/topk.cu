@@ -25,9 +25,13 @@ constexpr int kTopkChunkTarget = LOKI_TOPK_CHUNK_TARGET;
 // One CTA (or one cluster of CTAs) per row. CTA rank r of the row's cluster
 // holds keys [r * chunk, min((r + 1) * chunk, S)); chunk is a multiple of 4
 // and at most 4 * NT * I.
+// With lens (a per-sequence length, row r belonging to sequence r / H_q) a
+// row holds lens[r / H_q] <= S keys at stride S: it selects min(k, length)
+// and pads its output with -1.
 template <int NT, int I, bool kCl>
 __global__ void __launch_bounds__(NT) k_topk(const float* __restrict__ scores, int S, int k,
-                                             int chunk, int32_t* __restrict__ out, int vec4) {
+                                             int chunk, int32_t* __restrict__ out, int vec4,
+                                             const int* __restrict__ lens, int H_q) {
     __shared__ __align__(16) uint32_t scratch[kTkSmemWords];
     TkCluster<kCl> cl;
     cl.init();
@@ -40,8 +44,14 @@ __global__ void __launch_bounds__(NT) k_topk(const float* __restrict__ scores, i
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row = blockIdx.x / cl.size;
     const int base = cl.rank * chunk;
-    const int n = max(0, min(chunk, S - base));
+    const int S_row = lens != nullptr ? min(S, max(0, lens[row / H_q])) : S;
+    const int k_row = min(k, S_row);
+    const int n = max(0, min(chunk, S_row - base));
     const float* src = scores + row * S + base;
+    int32_t* o = out + row * k;
+    if (cl.rank == 0)
+        for (int x = k_row + (int)threadIdx.x; x < k; x += NT) o[x] = -1;  // padding
+    if (k_row == 0) return;  // an empty sequence (uniform over the cluster)
     uint4 v[I];
 #pragma unroll
     for (int i = 0; i < I; ++i) {
@@ -64,7 +74,7 @@ __global__ void __launch_bounds__(NT) k_topk(const float* __restrict__ scores, i
         for (int e = 0; e < 4; ++e)
             if (kk[e] != 0u) atomicAdd(&sm.hist1[kk[e] >> 21], 1u);
     }
-    tk_select<NT, I, kCl>(cl, v, base, k, out + row * k, sm);
+    tk_select<NT, I, kCl>(cl, v, base, k_row, o, sm);
 }
 
 // exclusive prefix sum over the block; `total` gets the block sum
@@ -178,7 +188,7 @@ __global__ void __launch_bounds__(512) k_topk_long(const float* __restrict__ sco
 
 template <int NT, int I, bool kCl>
 static cudaError_t launch_rows(const float* scores, int64_t rows, int S, int k, int C, int chunk,
-                               int32_t* idx, cudaStream_t s, bool pdl) {
+                               int32_t* idx, cudaStream_t s, bool pdl, const int* lens, int H_q) {
     auto kern = k_topk<NT, I, kCl>;
     cudaError_t e = prefer_carveout(reinterpret_cast<const void*>(kern),
                                     cudaSharedmemCarveoutMaxShared);
@@ -206,14 +216,16 @@ static cudaError_t launch_rows(const float* scores, int64_t rows, int S, int k, 
     }
     cfg.attrs = na ? attr : nullptr;
     cfg.numAttrs = (unsigned)na;
-    return cudaLaunchKernelEx(&cfg, kern, scores, S, k, chunk, idx, vec4);
+    return cudaLaunchKernelEx(&cfg, kern, scores, S, k, chunk, idx, vec4, lens, H_q);
 }
 
 template <bool kCl>
 static cudaError_t launch_shape(int nt, int gi, const float* scores, int64_t rows, int S, int k,
-                                int C, int chunk, int32_t* idx, cudaStream_t s, bool pdl) {
-#define LOKI_TK(NT_, I_) \
-    if (nt == NT_ && gi == I_) return launch_rows<NT_, I_, kCl>(scores, rows, S, k, C, chunk, idx, s, pdl);
+                                int C, int chunk, int32_t* idx, cudaStream_t s, bool pdl,
+                                const int* lens, int H_q) {
+#define LOKI_TK(NT_, I_)                                                                        \
+    if (nt == NT_ && gi == I_)                                                                  \
+        return launch_rows<NT_, I_, kCl>(scores, rows, S, k, C, chunk, idx, s, pdl, lens, H_q);
     LOKI_TK(128, 1) LOKI_TK(128, 2) LOKI_TK(128, 4)
     LOKI_TK(256, 4) LOKI_TK(256, 8) LOKI_TK(512, 8)
     LOKI_TK(256, 1) LOKI_TK(512, 1)
@@ -258,16 +270,19 @@ bool topk_shape(int64_t rows, int64_t S, int sm_count, int* C_out, int* chunk_ou
 }
 
 cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k, int32_t* idx,
-                        cudaStream_t s, bool pdl) {
+                        cudaStream_t s, bool pdl, const int* lens, int H_q) {
     const int Si = (int)S, ki = (int)k;
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     int C, chunk, nt, gi;
     if (topk_shape(rows, S, di.sm_count, &C, &chunk, &nt, &gi)) {
-        if (C == 1) return launch_shape<false>(nt, gi, scores, rows, Si, ki, 1, chunk, idx, s, pdl);
-        return launch_shape<true>(nt, gi, scores, rows, Si, ki, C, chunk, idx, s, pdl);
+        if (C == 1)
+            return launch_shape<false>(nt, gi, scores, rows, Si, ki, 1, chunk, idx, s, pdl, lens,
+                                       H_q);
+        return launch_shape<true>(nt, gi, scores, rows, Si, ki, C, chunk, idx, s, pdl, lens, H_q);
     }
+    if (lens != nullptr) return cudaErrorInvalidValue;  // per-row lengths: up to 262144 keys
     {
         const size_t need = (size_t)S * 4;
         if (need + 4096 <= (size_t)di.smem_optin) {

@@ -161,3 +161,44 @@ def test_fused_entry_point_rejects_bad_arguments(L):
     assert dec(H_q=3) == 1             # H_q not a multiple of H_kv
     assert dec(out=FAKE + 2) == 1      # misaligned output
     assert L.lib.loki_last_error().decode() != ""
+
+
+def test_paged_entry_points_reject_bad_arguments(L):
+    f = 1 << 20  # fake, 1 MiB-aligned device pointers (never dereferenced)
+    ws = L.lib.loki_paged_decode_workspace_size(2, 4, 4, 16, 8, 128, 32, 64)
+    assert ws > 0
+
+    def dec(page_size=16, max_pages=8, n_pages=20, d_lo=32, d=32, k=64, q=f, H_q=4, H_kv=4):
+        return L.lib.loki_decode_attention_paged(q, f, f, f, d_lo, f, f, f, 2, H_q, H_kv, page_size,
+                                                 max_pages, n_pages, 128, d, k, 0.0, L.DTYPE_BF16,
+                                                 f, f, f, ws, None)
+
+    assert dec(page_size=0) == 1
+    assert dec(n_pages=0) == 1
+    assert dec(d=40) == 1                     # d > d_lo
+    assert dec(k=16 * 8 + 1) == 1             # k beyond page_size * max_pages
+    assert dec(d_lo=128, d=32) == 2           # plane rows the paged scan does not take
+    assert dec(H_q=16, H_kv=2, d_lo=32) == 2  # G * d_lo > 64
+    assert dec(page_size=4096, max_pages=128, k=64) == 2  # more than 262144 tokens
+    assert dec(q=f + 2) == 1                  # misaligned
+    assert L.lib.loki_decode_attention_paged(f, f, f, f, 32, f, f, f, 2, 4, 4, 16, 8, 20, 128,
+                                             32, 64, 0.0, L.DTYPE_BF16, f, f, f, ws - 1, None) == 3
+    # the append
+    assert L.lib.loki_append_keys_paged(f, f, f, f, f, None, 0, f, f, 2, 4, 0, 16, 8, 20, 128,
+                                        L.DTYPE_BF16, None) == 1  # T = 0
+    assert L.lib.loki_append_keys_paged(f, f, f, f, f, f, 12, f, f, 2, 4, 1, 16, 8, 20, 128,
+                                        L.DTYPE_BF16, None) == 1  # plane row of 24 bytes
+    assert L.lib.loki_append_keys_paged(f, f, f, f, f, None, 0, f, f + 1, 2, 4, 1, 16, 8, 20, 128,
+                                        L.DTYPE_BF16, None) == 1  # misaligned positions
+
+
+def test_decode_step_rejects_bad_arguments_on_the_host(L):
+    f = 1 << 20
+    ws = L.lib.loki_decode_workspace_size(1, 2, 2, 64, 128, 32, 8)
+    # T = 0, a NULL new key, k > pos + T
+    assert L.lib.loki_decode_step(f, f, f, f, f, f, None, 0, 1, 2, 2, 0, 10, 64, 128, 32, 8, 0.0,
+                                  L.DTYPE_BF16, f, f, f, ws, None) == 1
+    assert L.lib.loki_decode_step(f, None, f, f, f, f, None, 0, 1, 2, 2, 1, 10, 64, 128, 32, 8,
+                                  0.0, L.DTYPE_BF16, f, f, f, ws, None) == 1
+    assert L.lib.loki_decode_step(f, f, f, f, f, f, None, 0, 1, 2, 2, 1, 2, 64, 128, 32, 8, 0.0,
+                                  L.DTYPE_BF16, f, f, f, ws, None) == 1
