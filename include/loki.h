@@ -337,6 +337,29 @@ LOKI_API loki_status loki_sparse_attention(const float* q_rot, const void* Kt_ca
                                   loki_dtype dt, void* out, void* ws, size_t ws_bytes,
                                   void* stream);
 
+/* PCAAttn ------------------------------------------------------------------ */
+
+/* Bytes of workspace loki_pca_attention needs (q~ and split-S partials). */
+LOKI_API size_t loki_pca_attention_workspace_size(int B, int H_q, int H_kv, int64_t S, int D);
+
+/*
+ * PCAAttn, the variant of Loki the poster page evaluates in its "More on
+ * tables" PCAAttn table: the softmax is taken directly over the
+ * reduced-dimensional scores of all S cached tokens, with no top-k and no
+ * full-dimensional rescoring:
+ *   s_j = q~[:d] . K~_j[:d] (q~ = q P), p = softmax(scale * s) over j < S,
+ *   out = sum_j p_j V_j.
+ * The keys are read from the low-dimensional key plane Kt_lo [B, H_kv, S_max,
+ * d_lo] (plane rows of 16, 32, 64 or 128 bytes, d <= d_lo), the values in
+ * full. scale <= 0 selects 1/sqrt(D) (the reading: the same scale as the full
+ * scores). Arithmetic: fp32.
+ */
+LOKI_API loki_status loki_pca_attention(const void* q, const void* Kt_lo, int d_lo,
+                                        const void* V_cache, const float* P, int B, int H_q,
+                                        int H_kv, int64_t S, int64_t S_max, int D, int d,
+                                        float scale, loki_dtype dt, void* out, void* ws,
+                                        size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Dense baseline                                                           */
 /* ------------------------------------------------------------------------ */

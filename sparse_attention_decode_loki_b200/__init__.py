@@ -24,7 +24,7 @@ __all__ = [
     "loki_calibrate_pca", "loki_append_keys", "loki_decode_attention", "dense_decode_attention",
     "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_fused",
     "loki_decode_step", "loki_decode_attention_paged", "loki_append_keys_paged",
-    "loki_paged_decode_workspace_size",
+    "loki_paged_decode_workspace_size", "loki_pca_attention", "loki_pca_attention_workspace_size",
     "loki_decode_attention_noalloc",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
@@ -486,6 +486,32 @@ def loki_sparse_attention(q_rot: torch.Tensor, Kt_cache: torch.Tensor, V_cache: 
                                     selected_idx.data_ptr(), B, H_q, H_kv, S, S_max, D, k,
                                     float(scale), _dt(Kt_cache), out.data_ptr(), ws.data_ptr(),
                                     _ws_bytes(ws), _stream(dev)), "loki_sparse_attention")
+    return out
+
+
+def loki_pca_attention_workspace_size(B: int, H_q: int, H_kv: int, S: int, D: int) -> int:
+    return int(lib.loki_pca_attention_workspace_size(B, H_q, H_kv, S, D))
+
+
+def loki_pca_attention(q: torch.Tensor, Kt_lo: torch.Tensor, V_cache: torch.Tensor,
+                       P: torch.Tensor, S: int, d: int, scale: float = 0.0,
+                       out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """PCAAttn: softmax over the d-dimensional scores of all S tokens (keys from
+    the key plane Kt_lo [B, H_kv, S_max, d_lo]), times the values."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q, V_cache, V_cache, P)
+    _check_plane(Kt_lo, V_cache)
+    if out is None:
+        out = torch.empty_like(q)
+    _cuda(q, out)
+    _expect(out, q.shape, q.dtype, "out")
+    if S > S_max:
+        raise ValueError("S must be <= S_max")
+    ws = _ws(loki_pca_attention_workspace_size(B, H_q, H_kv, S, D), dev, workspace)
+    check(lib.loki_pca_attention(q.data_ptr(), Kt_lo.data_ptr(), Kt_lo.shape[3],
+                                 V_cache.data_ptr(), P.data_ptr(), B, H_q, H_kv, S, S_max, D, d,
+                                 float(scale), _dt(q), out.data_ptr(), ws.data_ptr(),
+                                 _ws_bytes(ws), _stream(dev)), "loki_pca_attention")
     return out
 
 

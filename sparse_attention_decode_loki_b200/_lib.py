@@ -74,6 +74,10 @@ PROTOTYPES = {
     "loki_sparse_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                       c_int64, c_int64, c_int, c_int64, c_float, c_int, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
+    "loki_pca_attention_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int64, c_int]),
+    "loki_pca_attention": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
+                                   c_int, c_int64, c_int64, c_int, c_int, c_float, c_int,
+                                   c_void_p, c_void_p, c_size_t, c_void_p]),
     "dense_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int64, c_int]),
     "dense_decode_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int64,
                                        c_int64, c_int, c_float, c_int, c_void_p, c_void_p, c_size_t,

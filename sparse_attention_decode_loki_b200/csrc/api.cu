@@ -728,6 +728,44 @@ loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, cons
 
 // ---------------------------------------------------------------------------
 
+size_t loki_pca_attention_workspace_size(int B, int H_q, int H_kv, int64_t S, int D) {
+    (void)H_kv;
+    if (B < 1 || H_q < 1 || S < 1 || D < 1) return 0;
+    return align_up((size_t)B * H_q * D * sizeof(float)) + dense_ws(B, H_q, S, D).total;
+}
+
+loki_status loki_pca_attention(const void* q, const void* Kt_lo, int d_lo, const void* V_cache,
+                               const float* P, int B, int H_q, int H_kv, int64_t S,
+                               int64_t S_max, int D, int d, float scale, loki_dtype dt, void* out,
+                               void* ws, size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    LOKI_REQUIRE(d >= 1 && d <= d_lo, LOKI_ERR_INVALID_ARG, "d must be in [1, d_lo] (got %d)", d);
+    const loki::Dt t = to_dt(dt);
+    LOKI_REQUIRE(loki::pca_attention_supported(t, d_lo), LOKI_ERR_UNSUPPORTED,
+                 "PCAAttn takes plane rows of 16, 32, 64 or 128 bytes");
+    LOKI_PTR(q, 16);
+    LOKI_PTR(Kt_lo, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(ws, 256);
+    const size_t qbytes = align_up((size_t)B * H_q * D * sizeof(float));
+    const DenseWs w = dense_ws(B, H_q, S, D);
+    LOKI_REQUIRE(ws_bytes >= qbytes + w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, qbytes + w.total);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* q_rot = at<float>(ws, 0);
+    void* dws = at<char>(ws, qbytes);
+    LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), "loki_pca_attention");
+    LOKI_CUDA(loki::launch_pca_attention(t, q_rot, Kt_lo, d_lo, d, V_cache, B, H_q, H_kv, S, S_max,
+                                         resolve_scale(scale, D), out, at<float2>(dws, w.ml),
+                                         at<float>(dws, w.acc), s),
+              "loki_pca_attention");
+    return LOKI_OK;
+}
+
 size_t dense_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, int D) {
     (void)H_kv;
     if (B < 1 || H_q < 1 || S < 1 || D < 1) return 0;

@@ -9,6 +9,13 @@
 // rows in flight per group) and keeps an online softmax for each of the G
 // query heads of its KV head, so every key/value byte is read once for all G
 // heads. Partials are merged by k_combine.
+//
+// The same kernel computes PCAAttn, the variant of Loki that applies the
+// softmax directly to the reduced-dimensional scores of every token (poster
+// page, "More on tables", PCAAttn table caption): the key of token j is then
+// its row of the low-dimensional key plane (d_lo columns, read by the first
+// d_lo * elem / 16 lanes of the row group) and the query is q~[:d], so the
+// score is s_j = q~[:d] . K~_j[:d]; the values are read in full.
 #include "combine.cuh"
 #include "common.cuh"
 #include "launch.h"
@@ -20,8 +27,12 @@ constexpr int kDenseMinRows = 256;
 // per >= kDenseMinRows / 2 (see sparse_max_parts for the argument)
 int64_t dense_max_parts(int64_t S) { return (S - 1) / (kDenseMinRows / 2) + 2; }
 
-template <class E, int G>
+// NVK = 0: dense attention, keys are full rows and q is of type E::T.
+// NVK > 0: PCAAttn, keys are plane rows of NVK 16-byte chunks and the query is
+// q_rot (fp32 q~), of which the first d columns count.
+template <class E, int G, int NVK>
 __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__ q,
+                                               const float* __restrict__ q_rot, int d,
                                                const typename E::T* __restrict__ K,
                                                const typename E::T* __restrict__ V, int H_q,
                                                int H_kv, int S, int64_t S_max, float scale_log2,
@@ -34,12 +45,14 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
     constexpr int NGRP = 256 / LPR;
     constexpr int U = G <= 2 ? 4 : 2;
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
+    constexpr int64_t kKeyBytes = NVK == 0 ? kRowBytes : (int64_t)NVK * 16;
     __shared__ float sm_m[G][NGRP], sm_l[G][NGRP];
     __shared__ float sm_acc[NGRP][D];
 
     const int grp = threadIdx.x / LPR;
     const int sub = threadIdx.x % LPR;
     griddep_launch_dependents();  // lets the combine kernel be scheduled early
+    if constexpr (NVK > 0) griddep_wait();  // q~ comes from the projection kernel
 
     int64_t w = (int64_t)blockIdx.x * per;
     const int64_t w_end = min64(w + per, total);
@@ -52,12 +65,23 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
         float qv[G][KV];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const typename E::T* qp = q + ((int64_t)b * H_q + (int64_t)hk * G + g) * D + sub * KV;
+            const int64_t qr = (int64_t)b * H_q + (int64_t)hk * G + g;
+            if constexpr (NVK == 0) {
+                const typename E::T* qp = q + qr * D + sub * KV;
 #pragma unroll
-            for (int e = 0; e < KV; ++e) qv[g][e] = E::load1(qp + e) * scale_log2;
+                for (int e = 0; e < KV; ++e) qv[g][e] = E::load1(qp + e) * scale_log2;
+            } else {
+#pragma unroll
+                for (int e = 0; e < KV; ++e) {
+                    const int col = sub * KV + e;
+                    qv[g][e] = (sub < NVK && col < d) ? __ldg(q_rot + qr * D + col) * scale_log2
+                                                      : 0.f;
+                }
+            }
         }
-        const char* Kb =
-            reinterpret_cast<const char*>(K) + (unit * S_max + s0) * kRowBytes + sub * 16;
+        const bool k_lane = NVK == 0 || sub < NVK;  // this lane reads part of the key row
+        const char* Kb = reinterpret_cast<const char*>(K) + (unit * S_max + s0) * kKeyBytes +
+                         (k_lane ? sub * 16 : 0);
         const char* Vb =
             reinterpret_cast<const char*>(V) + (unit * S_max + s0) * kRowBytes + sub * 16;
 
@@ -78,7 +102,8 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
                 const int row = pb + u * NGRP + grp;
                 ok[u] = row < seg;
                 if (ok[u]) {
-                    kv[u] = ld_stream(Kb + (int64_t)row * kRowBytes);
+                    kv[u] = k_lane ? ld_stream(Kb + (int64_t)row * kKeyBytes)
+                                   : make_uint4(0u, 0u, 0u, 0u);
                     vv[u] = ld_stream(Vb + (int64_t)row * kRowBytes);
                 } else {
                     kv[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -153,15 +178,16 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
     }
 }
 
-template <class E, int G>
-static cudaError_t dense_impl(const void* q, const void* K, const void* V, int B, int H_q,
-                              int H_kv, int64_t S, int64_t S_max, int D, float scale, void* out,
-                              float2* part_ml, float* part_acc, cudaStream_t s) {
+template <class E, int G, int NVK>
+static cudaError_t dense_impl(const void* q, const float* q_rot, int d, const void* K,
+                              const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
+                              int D, float scale, void* out, float2* part_ml, float* part_acc,
+                              cudaStream_t s, bool pdl) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const int64_t total = (int64_t)B * H_kv * S;
-    auto kern = k_dense<E, G>;
+    auto kern = k_dense<E, G, NVK>;
     const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0);
     int64_t grid = (total + kDenseMinRows - 1) / kDenseMinRows;
     if (grid > resident) grid = resident;
@@ -170,29 +196,66 @@ static cudaError_t dense_impl(const void* q, const void* K, const void* V, int B
     const int maxp = (int)((S - 1) / per + 2);
     if (maxp > dense_max_parts(S)) return cudaErrorInvalidValue;
     using T = typename E::T;
-    kern<<<(unsigned)grid, 256, 0, s>>>(static_cast<const T*>(q), static_cast<const T*>(K),
-                                        static_cast<const T*>(V), H_q, H_kv, (int)S, S_max,
-                                        scale * kLog2e, total, per, maxp, part_ml, part_acc);
-    e = cudaGetLastError();
+    e = launch_kernel(kern, dim3((unsigned)grid), dim3(256), 0, s, pdl, static_cast<const T*>(q),
+                      q_rot, d, static_cast<const T*>(K), static_cast<const T*>(V), H_q, H_kv,
+                      (int)S, S_max, scale * kLog2e, total, per, maxp, part_ml, part_acc);
     if (e != cudaSuccess) return e;
     return launch_kernel(k_combine<E>, dim3((unsigned)((int64_t)B * H_q)), dim3(128), 0, s, true,
                          (const float2*)part_ml, (const float*)part_acc, static_cast<T*>(out), H_q,
                          G, (int64_t)S, per, maxp, D);
 }
 
-template <class E>
-static cudaError_t dense_dispatch(int G, const void* q, const void* K, const void* V, int B,
-                                  int H_q, int H_kv, int64_t S, int64_t S_max, int D, float scale,
-                                  void* out, float2* part_ml, float* part_acc, cudaStream_t s) {
+template <class E, int NVK>
+static cudaError_t dense_dispatch(int G, const void* q, const float* q_rot, int d, const void* K,
+                                  const void* V, int B, int H_q, int H_kv, int64_t S,
+                                  int64_t S_max, int D, float scale, void* out, float2* part_ml,
+                                  float* part_acc, cudaStream_t s, bool pdl) {
     switch (G) {
-#define LOKI_G(g)                                                                             \
-    case g:                                                                                   \
-        return dense_impl<E, g>(q, K, V, B, H_q, H_kv, S, S_max, D, scale, out, part_ml, \
-                                part_acc, s);
+#define LOKI_G(g)                                                                               \
+    case g:                                                                                     \
+        return dense_impl<E, g, NVK>(q, q_rot, d, K, V, B, H_q, H_kv, S, S_max, D, scale, out, \
+                                     part_ml, part_acc, s, pdl);
         LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
 #undef LOKI_G
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <class E>
+static cudaError_t pca_nvk(int nvk, int G, const float* q_rot, int d, const void* Klo,
+                           const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
+                           float scale, void* out, float2* part_ml, float* part_acc,
+                           cudaStream_t s) {
+    switch (nvk) {
+#define LOKI_NVK(n)                                                                            \
+    case n:                                                                                    \
+        return dense_dispatch<E, n>(G, nullptr, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, 128, \
+                                    scale, out, part_ml, part_acc, s, true);
+        LOKI_NVK(1) LOKI_NVK(2) LOKI_NVK(4) LOKI_NVK(8)
+#undef LOKI_NVK
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+bool pca_attention_supported(Dt dt, int d_lo) {
+    const int row_bytes = d_lo * (dt == kF32 ? 4 : 2);
+    const int nvk = row_bytes / 16;
+    return row_bytes % 16 == 0 && (nvk == 1 || nvk == 2 || nvk == 4 || nvk == 8) &&
+           nvk <= 128 / (dt == kF32 ? 4 : 8);
+}
+
+cudaError_t launch_pca_attention(Dt dt, const float* q_rot, const void* Klo, int d_lo, int d,
+                                 const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
+                                 float scale, void* out, float2* part_ml, float* part_acc,
+                                 cudaStream_t s) {
+    if (!pca_attention_supported(dt, d_lo)) return cudaErrorInvalidValue;
+    const int G = H_q / H_kv;
+    const int nvk = d_lo * (dt == kF32 ? 4 : 2) / 16;
+    if (dt == kF32)
+        return pca_nvk<ElemF32>(nvk, G, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, scale, out,
+                                part_ml, part_acc, s);
+    return pca_nvk<ElemBF16>(nvk, G, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, scale, out,
+                             part_ml, part_acc, s);
 }
 
 cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int B, int H_q,
@@ -200,10 +263,10 @@ cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int
                          float2* part_ml, float* part_acc, cudaStream_t s) {
     const int G = H_q / H_kv;
     if (dt == kF32)
-        return dense_dispatch<ElemF32>(G, q, K, V, B, H_q, H_kv, S, S_max, D, scale, out, part_ml,
-                                       part_acc, s);
-    return dense_dispatch<ElemBF16>(G, q, K, V, B, H_q, H_kv, S, S_max, D, scale, out, part_ml,
-                                    part_acc, s);
+        return dense_dispatch<ElemF32, 0>(G, q, nullptr, 128, K, V, B, H_q, H_kv, S, S_max, D,
+                                          scale, out, part_ml, part_acc, s, false);
+    return dense_dispatch<ElemBF16, 0>(G, q, nullptr, 128, K, V, B, H_q, H_kv, S, S_max, D, scale,
+                                       out, part_ml, part_acc, s, false);
 }
 
 }  // namespace loki

@@ -146,6 +146,15 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
                           int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl,
                           const PagedKV* pg = nullptr, const int* positions = nullptr);
 
+// PCAAttn: softmax over the low-dimensional scores s_j = q~[:d] . K~_j[:d] of
+// all S tokens (keys from the plane Klo [B, H_kv, S_max, d_lo]), out = sum p_j
+// V_j. A programmatic dependent of the projection that writes q_rot.
+bool pca_attention_supported(Dt dt, int d_lo);
+cudaError_t launch_pca_attention(Dt dt, const float* q_rot, const void* Klo, int d_lo, int d,
+                                 const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
+                                 float scale, void* out, float2* part_ml, float* part_acc,
+                                 cudaStream_t s);
+
 // ---- supporting subsystems -----------------------------------------------
 // Kt_lo (may be null): [B, H_kv, S_max, d_lo] plane that also receives the
 // first d_lo rotated columns of each appended key.
