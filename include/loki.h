@@ -30,8 +30,9 @@
  *   - Arguments are checked on the host before anything is enqueued; on any
  *     error nothing is launched and a loki_status other than LOKI_OK is
  *     returned. loki_last_error() then describes the failing argument.
- *   - D must be 128 (other head sizes return LOKI_ERR_UNSUPPORTED) and
- *     H_q / H_kv must be at most 8.
+ *   - D must be 128 or 96, the head sizes the Loki pages name (others return
+ *     LOKI_ERR_UNSUPPORTED), and H_q / H_kv must be at most 8.
+ *     loki_decode_attention_fused takes D = 128 only.
  *   - Entry points are thread-safe; calls on one stream are ordered.
  */
 #ifndef LOKI_H
@@ -53,7 +54,7 @@ extern "C" {
 typedef enum loki_status {
     LOKI_OK = 0,
     LOKI_ERR_INVALID_ARG = 1,         /* null pointer, bad size, misaligned pointer */
-    LOKI_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. D != 128) */
+    LOKI_ERR_UNSUPPORTED = 2,         /* valid but not implemented (e.g. D = 64) */
     LOKI_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size() figure */
     LOKI_ERR_CUDA = 4                 /* a CUDA runtime call or launch failed */
 } loki_status;
@@ -304,8 +305,9 @@ LOKI_API loki_status loki_project_query(const void* q, const float* P, int B, in
  * scores [B, H_q, S] fp32: s_j = sum_{i<d} q_rot[i] K~_j[i] for j < S. Only
  * the first d columns of each cached key are read; each KV head's rows are
  * read once for all of its query heads. Kt_cache rows hold D elements: the
- * rotated cache (D = 128) or a low-dimensional key plane (D = d_lo, with
- * D * sizeof(dt) a multiple of 16 bytes); 1 <= d <= D. q_rot is [B, H_q, 128].
+ * rotated cache of heads of D = 128 or 96 (q_rot is then [B, H_q, D]), or a
+ * low-dimensional key plane of 128-wide heads (any other D = d_lo, with
+ * D * sizeof(dt) a multiple of 16 bytes; q_rot is [B, H_q, 128]); 1 <= d <= D.
  */
 LOKI_API loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, int H_q, int H_kv,
                               int64_t S, int64_t S_max, int D, int d, loki_dtype dt,

@@ -424,15 +424,17 @@ def loki_score_lowdim(q_rot: torch.Tensor, Kt_cache: torch.Tensor, S: int, d: in
                       scores: Optional[torch.Tensor] = None) -> torch.Tensor:
     """fp32 scores [B, H_q, S] on the first d rotated dimensions.
 
-    Kt_cache is the rotated cache [B, H_kv, S_max, 128] or a low-dimensional
-    key plane [B, H_kv, S_max, d_lo]; its last dimension is the row width the
-    scan strides by.
+    Kt_cache is the rotated cache [B, H_kv, S_max, D] of heads of D = 128 or
+    96 (q_rot is then [B, H_q, D]), or a low-dimensional key plane
+    [B, H_kv, S_max, d_lo] of 128-wide heads (q_rot [B, H_q, 128]); its last
+    dimension is the row width the scan strides by.
     """
     dev = _cuda(q_rot, Kt_cache)
     B, H_q, Dq = q_rot.shape
     Bk, H_kv, S_max, row = Kt_cache.shape
-    if q_rot.dtype != torch.float32 or Dq != 128:
-        raise TypeError("q_rot must be float32 [B, H_q, 128]")
+    want = row if row in (96, 128) else 128
+    if q_rot.dtype != torch.float32 or Dq != want:
+        raise TypeError(f"q_rot must be float32 [B, H_q, {want}]")
     if Bk != B or not 1 <= d <= row or S > S_max:
         raise ValueError("Kt_cache must be [B, H_kv, S_max >= S, row >= d]")
     if scores is None:

@@ -55,7 +55,8 @@ loki_status check_heads(int B, int H_q, int H_kv, int D) {
     LOKI_REQUIRE(H_q / H_kv <= kMaxGroup, LOKI_ERR_UNSUPPORTED,
                  "H_q / H_kv = %d exceeds the supported group size %d", H_q / H_kv, kMaxGroup);
     LOKI_REQUIRE(D >= 1, LOKI_ERR_INVALID_ARG, "D must be >= 1");
-    LOKI_REQUIRE(D == 128, LOKI_ERR_UNSUPPORTED, "D = %d: only D = 128 is implemented", D);
+    LOKI_REQUIRE(D == 128 || D == 96, LOKI_ERR_UNSUPPORTED,
+                 "D = %d: head dimensions 128 and 96 are implemented", D);
     LOKI_REQUIRE((int64_t)B * H_q <= 0x7fffffff, LOKI_ERR_INVALID_ARG, "B * H_q too large");
     return LOKI_OK;
 }
@@ -542,8 +543,8 @@ loki_status loki_decode_attention_paged(const void* q, const void* Kt_pages, con
     LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s, done, rows), name);
     LOKI_CUDA(loki::launch_paged_prefix(seq_lens, B, H_kv, S_cap, start_ws, grid, s), name);
     LOKI_CUDA(loki::launch_score_paged(t, q_rot, Kt_lo_pages, d_lo, block_table, start_ws, B, H_q,
-                                       H_kv, page_size, max_pages, n_pages, S_cap, d, scores, grid,
-                                       s),
+                                       H_kv, page_size, max_pages, n_pages, S_cap, d, D, scores,
+                                       grid, s),
               name);
     const int* lens = loki::paged_lens(start_ws, B);
     LOKI_CUDA(loki::launch_topk(scores, (int64_t)rows, S_cap, k, selected_idx, s, true, lens, H_q),
@@ -645,9 +646,11 @@ loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, i
                               float* scores, void* stream) {
     g_last_error.clear();
     LOKI_CHECK(check_dtype(dt));
-    // Kt_cache rows hold D elements: the rotated cache (D = 128) or a
-    // low-dimensional key plane (D = d_lo); q_rot rows always hold 128.
-    LOKI_CHECK(check_heads(B, H_q, H_kv, 128));
+    // Kt_cache rows hold D elements: the rotated cache of 128- or 96-wide
+    // heads (D = 128 or 96, and q_rot rows hold D), or a low-dimensional key
+    // plane of 128-wide heads (any other D = d_lo; q_rot rows hold 128).
+    const int Dq = (D == 96 || D == 128) ? D : 128;
+    LOKI_CHECK(check_heads(B, H_q, H_kv, Dq));
     LOKI_CHECK(check_seq(S, S_max));
     LOKI_CHECK(check_plane(D, 128, dt));
     LOKI_REQUIRE(d >= 1 && d <= D, LOKI_ERR_INVALID_ARG, "d must be in [1, D] (got %d)", d);
@@ -656,13 +659,13 @@ loki_status loki_score_lowdim(const float* q_rot, const void* Kt_cache, int B, i
     LOKI_PTR(scores, 4);
     // a plane (row width < 128) goes through the same TMA-staged scan as the
     // decode step; the rotated cache through the register-staged scan
-    if (D < 128)
-        LOKI_CUDA(loki::launch_score_plane(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, 128,
+    if (D < Dq)
+        LOKI_CUDA(loki::launch_score_plane(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, Dq,
                                            D, d, scores, static_cast<cudaStream_t>(stream), false),
                   "loki_score_lowdim");
     else
-        LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max,
-                                            128, D, d, scores, static_cast<cudaStream_t>(stream),
+        LOKI_CUDA(loki::launch_score_lowdim(to_dt(dt), q_rot, Kt_cache, B, H_q, H_kv, S, S_max, Dq,
+                                            D, d, scores, static_cast<cudaStream_t>(stream),
                                             false),
                   "loki_score_lowdim");
     return LOKI_OK;
@@ -760,7 +763,7 @@ loki_status loki_pca_attention(const void* q, const void* Kt_lo, int d_lo, const
     void* dws = at<char>(ws, qbytes);
     LOKI_CUDA(loki::launch_project_query(t, q, P, B, H_q, H_kv, D, q_rot, s), "loki_pca_attention");
     LOKI_CUDA(loki::launch_pca_attention(t, q_rot, Kt_lo, d_lo, d, V_cache, B, H_q, H_kv, S, S_max,
-                                         resolve_scale(scale, D), out, at<float2>(dws, w.ml),
+                                         D, resolve_scale(scale, D), out, at<float2>(dws, w.ml),
                                          at<float>(dws, w.acc), s),
               "loki_pca_attention");
     return LOKI_OK;

@@ -30,7 +30,9 @@ int64_t dense_max_parts(int64_t S) { return (S - 1) / (kDenseMinRows / 2) + 2; }
 // NVK = 0: dense attention, keys are full rows and q is of type E::T.
 // NVK > 0: PCAAttn, keys are plane rows of NVK 16-byte chunks and the query is
 // q_rot (fp32 q~), of which the first d columns count.
-template <class E, int G, int NVK>
+// DH: head dimension (96 or 128). The lanes keep the layout of 128 columns;
+// those past DH load nothing and write nothing.
+template <class E, int G, int NVK, int DH>
 __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__ q,
                                                const float* __restrict__ q_rot, int d,
                                                const typename E::T* __restrict__ K,
@@ -39,18 +41,19 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
                                                int64_t total, int64_t per, int maxp,
                                                float2* __restrict__ part_ml,
                                                float* __restrict__ part_acc) {
-    constexpr int D = 128;
+    constexpr int D = DH;
     constexpr int KV = E::kVec;
-    constexpr int LPR = D / KV;
+    constexpr int LPR = 128 / KV;
     constexpr int NGRP = 256 / LPR;
     constexpr int U = G <= 2 ? 4 : 2;
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
     constexpr int64_t kKeyBytes = NVK == 0 ? kRowBytes : (int64_t)NVK * 16;
     __shared__ float sm_m[G][NGRP], sm_l[G][NGRP];
-    __shared__ float sm_acc[NGRP][D];
+    __shared__ float sm_acc[NGRP][128];
 
     const int grp = threadIdx.x / LPR;
     const int sub = threadIdx.x % LPR;
+    const bool lane_on = sub * KV < D;
     griddep_launch_dependents();  // lets the combine kernel be scheduled early
     if constexpr (NVK > 0) griddep_wait();  // q~ comes from the projection kernel
 
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
             if constexpr (NVK == 0) {
                 const typename E::T* qp = q + qr * D + sub * KV;
 #pragma unroll
-                for (int e = 0; e < KV; ++e) qv[g][e] = E::load1(qp + e) * scale_log2;
+                for (int e = 0; e < KV; ++e) qv[g][e] = lane_on ? E::load1(qp + e) * scale_log2 : 0.f;
             } else {
 #pragma unroll
                 for (int e = 0; e < KV; ++e) {
@@ -79,11 +82,12 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
                 }
             }
         }
-        const bool k_lane = NVK == 0 || sub < NVK;  // this lane reads part of the key row
+        // this lane reads part of the key row
+        const bool k_lane = NVK == 0 ? lane_on : sub < NVK;
         const char* Kb = reinterpret_cast<const char*>(K) + (unit * S_max + s0) * kKeyBytes +
                          (k_lane ? sub * 16 : 0);
-        const char* Vb =
-            reinterpret_cast<const char*>(V) + (unit * S_max + s0) * kRowBytes + sub * 16;
+        const char* Vb = reinterpret_cast<const char*>(V) + (unit * S_max + s0) * kRowBytes +
+                         (lane_on ? sub * 16 : 0);
 
         float m[G], l[G], acc[G][KV];
 #pragma unroll
@@ -104,7 +108,8 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
                 if (ok[u]) {
                     kv[u] = k_lane ? ld_stream(Kb + (int64_t)row * kKeyBytes)
                                    : make_uint4(0u, 0u, 0u, 0u);
-                    vv[u] = ld_stream(Vb + (int64_t)row * kRowBytes);
+                    vv[u] = lane_on ? ld_stream(Vb + (int64_t)row * kRowBytes)
+                                    : make_uint4(0u, 0u, 0u, 0u);
                 } else {
                     kv[u] = make_uint4(0u, 0u, 0u, 0u);
                     vv[u] = kv[u];
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(256) k_dense(const typename E::T* __restrict__
     }
 }
 
-template <class E, int G, int NVK>
+template <class E, int G, int NVK, int DH>
 static cudaError_t dense_impl(const void* q, const float* q_rot, int d, const void* K,
                               const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
                               int D, float scale, void* out, float2* part_ml, float* part_acc,
@@ -187,7 +192,7 @@ static cudaError_t dense_impl(const void* q, const float* q_rot, int d, const vo
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const int64_t total = (int64_t)B * H_kv * S;
-    auto kern = k_dense<E, G, NVK>;
+    auto kern = k_dense<E, G, NVK, DH>;
     const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, 256, 0);
     int64_t grid = (total + kDenseMinRows - 1) / kDenseMinRows;
     if (grid > resident) grid = resident;
@@ -205,7 +210,7 @@ static cudaError_t dense_impl(const void* q, const float* q_rot, int d, const vo
                          G, (int64_t)S, per, maxp, D);
 }
 
-template <class E, int NVK>
+template <class E, int NVK, int DH>
 static cudaError_t dense_dispatch(int G, const void* q, const float* q_rot, int d, const void* K,
                                   const void* V, int B, int H_q, int H_kv, int64_t S,
                                   int64_t S_max, int D, float scale, void* out, float2* part_ml,
@@ -213,24 +218,24 @@ static cudaError_t dense_dispatch(int G, const void* q, const float* q_rot, int 
     switch (G) {
 #define LOKI_G(g)                                                                               \
     case g:                                                                                     \
-        return dense_impl<E, g, NVK>(q, q_rot, d, K, V, B, H_q, H_kv, S, S_max, D, scale, out, \
-                                     part_ml, part_acc, s, pdl);
+        return dense_impl<E, g, NVK, DH>(q, q_rot, d, K, V, B, H_q, H_kv, S, S_max, D, scale, \
+                                         out, part_ml, part_acc, s, pdl);
         LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
 #undef LOKI_G
         default: return cudaErrorInvalidValue;
     }
 }
 
-template <class E>
+template <class E, int DH>
 static cudaError_t pca_nvk(int nvk, int G, const float* q_rot, int d, const void* Klo,
                            const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
                            float scale, void* out, float2* part_ml, float* part_acc,
                            cudaStream_t s) {
     switch (nvk) {
-#define LOKI_NVK(n)                                                                            \
-    case n:                                                                                    \
-        return dense_dispatch<E, n>(G, nullptr, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, 128, \
-                                    scale, out, part_ml, part_acc, s, true);
+#define LOKI_NVK(n)                                                                          \
+    case n:                                                                                  \
+        return dense_dispatch<E, n, DH>(G, nullptr, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, \
+                                        DH, scale, out, part_ml, part_acc, s, true);
         LOKI_NVK(1) LOKI_NVK(2) LOKI_NVK(4) LOKI_NVK(8)
 #undef LOKI_NVK
         default: return cudaErrorInvalidValue;
@@ -246,27 +251,29 @@ bool pca_attention_supported(Dt dt, int d_lo) {
 
 cudaError_t launch_pca_attention(Dt dt, const float* q_rot, const void* Klo, int d_lo, int d,
                                  const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
-                                 float scale, void* out, float2* part_ml, float* part_acc,
+                                 int D, float scale, void* out, float2* part_ml, float* part_acc,
                                  cudaStream_t s) {
-    if (!pca_attention_supported(dt, d_lo)) return cudaErrorInvalidValue;
+    if (!pca_attention_supported(dt, d_lo) || (D != 96 && D != 128)) return cudaErrorInvalidValue;
     const int G = H_q / H_kv;
     const int nvk = d_lo * (dt == kF32 ? 4 : 2) / 16;
-    if (dt == kF32)
-        return pca_nvk<ElemF32>(nvk, G, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, scale, out,
-                                part_ml, part_acc, s);
-    return pca_nvk<ElemBF16>(nvk, G, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, scale, out,
-                             part_ml, part_acc, s);
+#define LOKI_PCA(E, DH) \
+    pca_nvk<E, DH>(nvk, G, q_rot, d, Klo, V, B, H_q, H_kv, S, S_max, scale, out, part_ml, part_acc, s)
+    if (dt == kF32) return D == 96 ? LOKI_PCA(ElemF32, 96) : LOKI_PCA(ElemF32, 128);
+    return D == 96 ? LOKI_PCA(ElemBF16, 96) : LOKI_PCA(ElemBF16, 128);
+#undef LOKI_PCA
 }
 
 cudaError_t launch_dense(Dt dt, const void* q, const void* K, const void* V, int B, int H_q,
                          int H_kv, int64_t S, int64_t S_max, int D, float scale, void* out,
                          float2* part_ml, float* part_acc, cudaStream_t s) {
     const int G = H_q / H_kv;
-    if (dt == kF32)
-        return dense_dispatch<ElemF32, 0>(G, q, nullptr, 128, K, V, B, H_q, H_kv, S, S_max, D,
-                                          scale, out, part_ml, part_acc, s, false);
-    return dense_dispatch<ElemBF16, 0>(G, q, nullptr, 128, K, V, B, H_q, H_kv, S, S_max, D, scale,
-                                       out, part_ml, part_acc, s, false);
+    if (D != 96 && D != 128) return cudaErrorInvalidValue;
+#define LOKI_DENSE(E, DH)                                                                         \
+    dense_dispatch<E, 0, DH>(G, q, nullptr, 128, K, V, B, H_q, H_kv, S, S_max, D, scale, out, \
+                             part_ml, part_acc, s, false)
+    if (dt == kF32) return D == 96 ? LOKI_DENSE(ElemF32, 96) : LOKI_DENSE(ElemF32, 128);
+    return D == 96 ? LOKI_DENSE(ElemBF16, 96) : LOKI_DENSE(ElemBF16, 128);
+#undef LOKI_DENSE
 }
 
 }  // namespace loki

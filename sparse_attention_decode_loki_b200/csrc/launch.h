@@ -123,7 +123,8 @@ const int* paged_lens(const void* start_ws, int B);
 cudaError_t launch_score_paged(Dt dt, const float* q_rot, const void* Klo_pages, int d_lo,
                                const int* block_table, const void* start_ws, int B, int H_q,
                                int H_kv, int page_size, int max_pages, int64_t n_pages,
-                               int64_t S_cap, int d, float* scores, int grid, cudaStream_t s);
+                               int64_t S_cap, int d, int D, float* scores, int grid,
+                               cudaStream_t s);
 
 // split-S partial slots per (batch, KV head) unit
 int64_t dense_max_parts(int64_t S);
@@ -152,7 +153,7 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
 bool pca_attention_supported(Dt dt, int d_lo);
 cudaError_t launch_pca_attention(Dt dt, const float* q_rot, const void* Klo, int d_lo, int d,
                                  const void* V, int B, int H_q, int H_kv, int64_t S, int64_t S_max,
-                                 float scale, void* out, float2* part_ml, float* part_acc,
+                                 int D, float scale, void* out, float2* part_ml, float* part_acc,
                                  cudaStream_t s);
 
 // ---- supporting subsystems -----------------------------------------------

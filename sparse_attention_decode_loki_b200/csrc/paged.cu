@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kPgThreads, 1) k_score_paged(
     const int* __restrict__ block_table, const int* __restrict__ lens,
     const PagedStart* __restrict__ starts, float* __restrict__ scores, int* __restrict__ err,
     int B, int H_q, int H_kv, int page_size, int max_pages, int64_t n_pages, int64_t S_cap,
-    int d) {
+    int d, int D) {
     constexpr int KV = E::kVec;
     constexpr int kRowBytes = NV * 16;
     constexpr int kTR = kPgConsumers;  // rows per tile
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kPgThreads, 1) k_score_paged(
         for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int x = 0; x < NV * KV; ++x)
-                qv[g][x] = x < d ? __ldcg(q_rot + (qrow0 + g) * 128 + x) : 0.f;
+                qv[g][x] = x < d ? __ldcg(q_rot + (qrow0 + g) * D + x) : 0.f;
         float* srow = scores + qrow0 * S_cap + c.j;
         for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
             const int n = min(kTR, seg - t0);
@@ -284,7 +284,7 @@ template <class E, int G, int NV>
 static cudaError_t paged_impl(const float* q_rot, const void* Klo, const int* bt, const int* lens,
                               const void* starts, float* scores, int* err, int B, int H_q,
                               int H_kv, int page_size, int max_pages, int64_t n_pages,
-                              int64_t S_cap, int d, int grid, cudaStream_t s) {
+                              int64_t S_cap, int d, int D, int grid, cudaStream_t s) {
     constexpr int kTile = kPgConsumers * NV * 16;
     constexpr int kStages = (kPgRingBytes / kTile) < kPgMaxStages ? (kPgRingBytes / kTile)
                                                                   : kPgMaxStages;
@@ -303,20 +303,20 @@ static cudaError_t paged_impl(const float* q_rot, const void* Klo, const int* bt
     return launch_kernel(kern, dim3((unsigned)grid), dim3(kPgThreads), smem, s, true, q_rot,
                          static_cast<const T*>(Klo), bt, lens,
                          static_cast<const PagedStart*>(starts), scores, err, B, H_q, H_kv,
-                         page_size, max_pages, n_pages, S_cap, d);
+                         page_size, max_pages, n_pages, S_cap, d, D);
 }
 
 template <class E, int G>
 static cudaError_t paged_nv(int nv, const float* q_rot, const void* Klo, const int* bt,
                             const int* lens, const void* starts, float* scores, int* err, int B,
                             int H_q, int H_kv, int page_size, int max_pages, int64_t n_pages,
-                            int64_t S_cap, int d, int grid, cudaStream_t s) {
+                            int64_t S_cap, int d, int D, int grid, cudaStream_t s) {
     switch (nv) {
 #define LOKI_NV(n)                                                                              \
     case n:                                                                                     \
         if constexpr (G * n * E::kVec <= 64)                                                    \
             return paged_impl<E, G, n>(q_rot, Klo, bt, lens, starts, scores, err, B, H_q, H_kv, \
-                                       page_size, max_pages, n_pages, S_cap, d, grid, s);       \
+                                       page_size, max_pages, n_pages, S_cap, d, D, grid, s);    \
         return cudaErrorInvalidValue;
         LOKI_NV(1) LOKI_NV(2) LOKI_NV(4) LOKI_NV(8)
 #undef LOKI_NV
@@ -351,7 +351,8 @@ const int* paged_lens(const void* start_ws, int B) {
 cudaError_t launch_score_paged(Dt dt, const float* q_rot, const void* Klo_pages, int d_lo,
                                const int* block_table, const void* start_ws, int B, int H_q,
                                int H_kv, int page_size, int max_pages, int64_t n_pages,
-                               int64_t S_cap, int d, float* scores, int grid, cudaStream_t s) {
+                               int64_t S_cap, int d, int D, float* scores, int grid,
+                               cudaStream_t s) {
     int* err = device_error_word();
     if (err == nullptr) return cudaErrorInvalidDevice;
     const int G = H_q / H_kv;
@@ -367,10 +368,10 @@ cudaError_t launch_score_paged(Dt dt, const float* q_rot, const void* Klo_pages,
         if (dt == kF32)                                                                        \
             return paged_nv<ElemF32, g>(nv, q_rot, Klo_pages, block_table, lens, starts,       \
                                         scores, err, B, H_q, H_kv, page_size, max_pages,       \
-                                        n_pages, S_cap, d, grid, s);                           \
+                                        n_pages, S_cap, d, D, grid, s);                        \
         return paged_nv<ElemBF16, g>(nv, q_rot, Klo_pages, block_table, lens, starts, scores,   \
                                      err, B, H_q, H_kv, page_size, max_pages, n_pages, S_cap,  \
-                                     d, grid, s);
+                                     d, D, grid, s);
         LOKI_G(1) LOKI_G(2) LOKI_G(3) LOKI_G(4) LOKI_G(5) LOKI_G(6) LOKI_G(7) LOKI_G(8)
 #undef LOKI_G
         default: return cudaErrorInvalidValue;

@@ -61,16 +61,17 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // row j of the chunk: sequence b = (r0 + j) / R, member g = (r0 + j) % R
-    // (a query head for g < G, else new key g - G); 8 elements per thread and step
+    // (a query head for g < G, else new key g - G); 8 elements per thread and
+    // step, in a layout of 128 columns whose columns past D stay zero
     constexpr int QV = 8;
     float xv[kRotRows * 128 / 256];
 #pragma unroll
     for (int u = 0; u < kRotRows * 128 / 256 / QV; ++u) {
         const int it = (tid + u * 256) * QV;
-        const int j = it / D, i = it % D;
+        const int j = it / 128, i = it % 128;
         const int64_t jr = r0 + j;
         const Tp* src = nullptr;
-        if (j < nrows) {
+        if (j < nrows && i < D) {
             const int b = (int)(jr / R), g = (int)(jr % R);
             src = g < G ? q + ((int64_t)b * H_q + (int64_t)hk * G + g) * D
                         : K_new + (((int64_t)b * H_kv + hk) * T + (g - G)) * D;
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
 #pragma unroll
     for (int u = 0; u < kRotRows * 128 / 256 / QV; ++u) {
         const int it = (tid + u * 256) * QV;
-        const int j = it / D, i = it % D;
+        const int j = it / 128, i = it % 128;
 #pragma unroll
         for (int e = 0; e < QV; ++e) xs[j][i + e] = xv[u * QV + e];
     }

@@ -45,17 +45,18 @@ __device__ __forceinline__ int64_t owner_warp(int64_t b, int64_t W, int64_t N) {
 
 // Issue the key and value loads of one batch: U rows per row group, rows
 // jb + u * GPW + grp of the staged index list (indices past n, or -1 for an
-// index outside [0, S), load nothing and give zeros).
+// index outside [0, S), load nothing and give zeros; so do lanes past the
+// head dimension).
 template <int U, int GPW>
 __device__ __forceinline__ void sp_load(const int* widx, int n, int jb, int grp, const char* Kb,
-                                        const char* Vb, int64_t row_bytes, int (&t)[U],
-                                        uint4 (&kv)[U], uint4 (&vv)[U]) {
+                                        const char* Vb, int64_t row_bytes, bool lane_on,
+                                        int (&t)[U], uint4 (&kv)[U], uint4 (&vv)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int jj = jb + u * GPW + grp;
         const int tok = jj < n ? widx[jj] : -1;
         t[u] = tok;
-        if (tok >= 0) {
+        if (tok >= 0 && lane_on) {
             kv[u] = ld_stream(Kb + (int64_t)tok * row_bytes);
             vv[u] = ld_stream(Vb + (int64_t)tok * row_bytes);
         } else {
@@ -102,34 +103,32 @@ __device__ __forceinline__ void sp_consume(const float (&qv)[E::kVec], const int
     m = mx;
 }
 
-#ifndef LOKI_SP_PIPE
-#define LOKI_SP_PIPE 0
-#endif
-#ifndef LOKI_SP_U
-#define LOKI_SP_U 8
-#endif
-#ifndef LOKI_SP_MINB
-#define LOKI_SP_MINB 2
-#endif
+// rows in flight per row group, resident CTAs per SM (measured: more CTAs
+// with fewer rows each, or two batches in flight per warp, are no faster)
+constexpr int kSpU = 8;
+constexpr int kSpMinBlocks = 2;
 
-template <class E>
-__global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
+// DH: head dimension (96 or 128). The lanes keep the layout of 128 columns;
+// those past DH load nothing and write nothing.
+template <class E, int DH>
+__global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int nblk, int64_t N, int64_t W,
     float2* __restrict__ part_ml, float* __restrict__ part_acc, int* __restrict__ done,
     typename E::T* __restrict__ out, const int* __restrict__ block_table, int page_size,
     int max_pages, int64_t n_pages, const int* __restrict__ lens, int* __restrict__ err) {
-    constexpr int D = 128;
+    constexpr int D = DH;
     constexpr int KV = E::kVec;
-    constexpr int LPR = D / KV;     // lanes per row
+    constexpr int LPR = 128 / KV;   // lanes per row
     constexpr int GPW = 32 / LPR;   // row groups per warp
-    constexpr int U = LOKI_SP_U;    // rows in flight per group
+    constexpr int U = kSpU;         // rows in flight per group
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
     __shared__ int s_idx[8][kWarpIdx];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / LPR, sub = lane % LPR;
+    const bool lane_on = sub * KV < D;
     const int G = H_q / H_kv;
     int* widx = s_idx[warp];
     griddep_wait();  // q_rot and the selected indices come from earlier kernels
@@ -152,7 +151,7 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
         {
             const float* qp = q_rot + r * D + sub * KV;
 #pragma unroll
-            for (int e = 0; e < KV; ++e) qv[e] = __ldg(qp + e) * scale_log2;
+            for (int e = 0; e < KV; ++e) qv[e] = lane_on ? __ldg(qp + e) * scale_log2 : 0.f;
         }
         // contiguous cache: rows of the unit; paged: rows of the page pool
         const int64_t base_row = block_table != nullptr ? 0 : unit * S_max;
@@ -195,27 +194,12 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
                 }
             }
             __syncwarp();
-#if LOKI_SP_PIPE
-            // two batches in registers: the next batch's loads are in flight
-            // while the current one is folded in
-            constexpr int STEP = GPW * U;
-            int tA[U], tB[U];
-            uint4 kA[U], vA[U], kB[U], vB[U];
-            sp_load<U, GPW>(widx, n, 0, grp, Kb, Vb, kRowBytes, tA, kA, vA);
-            for (int jb = 0; jb < n; jb += 2 * STEP) {
-                sp_load<U, GPW>(widx, n, jb + STEP, grp, Kb, Vb, kRowBytes, tB, kB, vB);
-                sp_consume<E, U, LPR>(qv, tA, kA, vA, m, l, acc);
-                sp_load<U, GPW>(widx, n, jb + 2 * STEP, grp, Kb, Vb, kRowBytes, tA, kA, vA);
-                sp_consume<E, U, LPR>(qv, tB, kB, vB, m, l, acc);
-            }
-#else
             for (int jb = 0; jb < n; jb += GPW * U) {
                 int t[U];
                 uint4 kv[U], vv[U];
-                sp_load<U, GPW>(widx, n, jb, grp, Kb, Vb, kRowBytes, t, kv, vv);
+                sp_load<U, GPW>(widx, n, jb, grp, Kb, Vb, kRowBytes, lane_on, t, kv, vv);
                 sp_consume<E, U, LPR>(qv, t, kv, vv, m, l, acc);
             }
-#endif
         }
         // merge the warp's row groups (lane l and lane l + LPR hold the same columns)
 #pragma unroll
@@ -236,7 +220,7 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
         const int64_t wf = owner_warp(r * nblk, W, N);
         const int64_t wl = owner_warp((r + 1) * nblk - 1, W, N);
         if (wf == wl) {  // the whole row is this warp's: normalise and write it
-            if (grp == 0) {
+            if (grp == 0 && lane_on) {
                 const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
                 for (int e = 0; e < KV; ++e) out[r * D + sub * KV + e] = E::from_float(acc[e] * inv);
@@ -244,7 +228,7 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
             continue;
         }
         const int64_t slot = r + w;
-        if (grp == 0) {
+        if (grp == 0 && lane_on) {
             float* pa = part_acc + slot * D + sub * KV;
 #pragma unroll
             for (int e = 0; e < KV; e += 4)
@@ -281,7 +265,9 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
 #pragma unroll 8
                 for (int p = 0; p < nparts; ++p) {
                     const float sc = exp2f(__ldcg(&ml[p].x) - M);
-                    const float4 a = __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane);
+                    const float4 a = 4 * lane < D ? __ldcg(reinterpret_cast<const float4*>(
+                                                        pacc + (int64_t)p * D) + lane)
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
                     A.x = fmaf(a.x, sc, A.x);
                     A.y = fmaf(a.y, sc, A.y);
                     A.z = fmaf(a.z, sc, A.z);
@@ -291,17 +277,19 @@ __global__ void __launch_bounds__(256, LOKI_SP_MINB) k_sparse_attn(
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
             const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-            typename E::T* o = out + r * D + 4 * lane;
-            o[0] = E::from_float(A.x * inv);
-            o[1] = E::from_float(A.y * inv);
-            o[2] = E::from_float(A.z * inv);
-            o[3] = E::from_float(A.w * inv);
+            if (4 * lane < D) {
+                typename E::T* o = out + r * D + 4 * lane;
+                o[0] = E::from_float(A.x * inv);
+                o[1] = E::from_float(A.y * inv);
+                o[2] = E::from_float(A.z * inv);
+                o[3] = E::from_float(A.w * inv);
+            }
             if (lane == 0) done[r] = 0;  // leave the counter ready for the next call
         }
     }
 }
 
-template <class E>
+template <class E, int DH>
 static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V,
                                const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                int64_t S_max, int D, int64_t k, float scale, void* out,
@@ -311,7 +299,7 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)B * H_q;
-    auto kern = k_sparse_attn<E>;
+    auto kern = k_sparse_attn<E, DH>;
     // the gathers in flight live in L1: the smallest shared split that still
     // holds two CTAs' staged indices (8 KB each, plus 1 KB reserved per CTA)
     const int pct = (2 * (8 + 1) * 1024 * 100 + di.smem_optin - 1) / di.smem_optin + 1;
@@ -341,11 +329,17 @@ cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, c
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
                                     float2* part_ml, float* part_acc, int* done, cudaStream_t s,
                                     bool pdl, const PagedKV& pg) {
+    if (D != 96 && D != 128) return cudaErrorInvalidValue;
     if (dt == kF32)
-        return sparse_impl<ElemF32>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                    part_ml, part_acc, done, s, pdl, pg);
-    return sparse_impl<ElemBF16>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k, scale, out,
-                                 part_ml, part_acc, done, s, pdl, pg);
+        return D == 96 ? sparse_impl<ElemF32, 96>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
+                                                  scale, out, part_ml, part_acc, done, s, pdl, pg)
+                       : sparse_impl<ElemF32, 128>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D,
+                                                   k, scale, out, part_ml, part_acc, done, s, pdl,
+                                                   pg);
+    return D == 96 ? sparse_impl<ElemBF16, 96>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
+                                               scale, out, part_ml, part_acc, done, s, pdl, pg)
+                   : sparse_impl<ElemBF16, 128>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
+                                                scale, out, part_ml, part_acc, done, s, pdl, pg);
 }
 
 }  // namespace loki
