@@ -362,6 +362,48 @@ LOKI_API loki_status loki_pca_attention(const void* q, const void* Kt_lo, int d_
                                         float scale, loki_dtype dt, void* out, void* ws,
                                         size_t ws_bytes, void* stream);
 
+/* Pre-rotary PCA ------------------------------------------------------------ */
+
+/*
+ * The pre-rotary variant the poster page compares with the post-rotary one
+ * ("More on figures": the perplexity figure with pre- and post-rotary PCA
+ * transforms, and the rank figure over pre- and post-rotary keys). The pages
+ * give no mechanism; the reading taken here: the basis P is calibrated on
+ * keys before the rotary position embedding, the token scores and the top-k
+ * use the pre-rotary query and keys in that basis, and the exact attention
+ * over the selected tokens uses the post-rotary query and keys, as the model
+ * would without Loki:
+ *   q~ = q_pre P, s_j = q~[:d] . K~pre_j[:d], I = top-k of s (ties to the
+ *   lower index, ascending), a_j = scale q_post . K_j for j in I,
+ *   out = softmax(a) V_I.
+ * The caches: Kt_lo [B, H_kv, S_max, d_lo] holds the first d_lo columns of
+ * the pre-rotary keys rotated by P (K_pre P, rounded once to dt); K_cache
+ * [B, H_kv, S_max, D] holds the post-rotary keys as the model makes them (in
+ * no PCA basis); V_cache the values. q_pre, q_post [B, H_q, D] of type dt.
+ * Workspace: loki_decode_prerotary_workspace_size bytes. Other arguments,
+ * limits and errors as loki_decode_attention_plane.
+ */
+LOKI_API size_t loki_decode_prerotary_workspace_size(int B, int H_q, int H_kv, int64_t S, int D,
+                                                     int d, int64_t k);
+LOKI_API loki_status loki_decode_attention_prerotary(
+    const void* q_pre, const void* q_post, const void* K_cache, const void* V_cache,
+    const void* Kt_lo, int d_lo, const float* P, int B, int H_q, int H_kv, int64_t S,
+    int64_t S_max, int D, int d, int64_t k, float scale, loki_dtype dt, void* out,
+    int32_t* selected_idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The append of the pre-rotary variant: T new tokens per (batch, KV head) at
+ * rows [pos, pos + T). The plane Kt_lo receives the first d_lo columns of
+ * K_new_pre P (pre-rotary keys [B, H_kv, T, D], rounded once to dt); K_cache
+ * receives K_new_post (the post-rotary keys) and V_cache V_new unchanged.
+ * Two kernels on `stream`; errors as loki_append_keys_plane.
+ */
+LOKI_API loki_status loki_append_keys_prerotary(const void* K_new_pre, const void* K_new_post,
+                                                const void* V_new, const float* P, void* K_cache,
+                                                void* V_cache, void* Kt_lo, int d_lo, int B,
+                                                int H_kv, int T, int D, int64_t S_max, int64_t pos,
+                                                loki_dtype dt, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Dense baseline                                                           */
 /* ------------------------------------------------------------------------ */

@@ -38,4 +38,5 @@ from .loki import (  # noqa: F401
     loki_decode,
     dense_decode,
     pca_attn_row,
+    prerotary_decode_row,
 )

@@ -209,6 +209,25 @@ def pca_attn_row(q: np.ndarray, Kt: np.ndarray, V: np.ndarray, P: np.ndarray, d:
     return (p @ np.asarray(V, dtype=np.float64)) / np.sum(p)
 
 
+def prerotary_decode_row(q_pre: np.ndarray, q_post: np.ndarray, Kt_pre: np.ndarray,
+                         K_post: np.ndarray, V: np.ndarray, P: np.ndarray, d: int, k: int,
+                         scale: float):
+    """Pre-rotary variant: select on the pre-rotary keys, attend on the post-rotary ones.
+
+    Poster page, "More on figures": the perplexity figure compares PCA
+    transforms of pre- and post-rotary keys, and the rank figure shows both
+    kinds of keys are low-rank. The pages give no mechanism; the reading: the
+    basis P comes from pre-rotary keys, so the scores and the top-k take the
+    pre-rotary query and keys in that basis (Kt_pre = K_pre P as cached), and
+    the exact attention over the selected tokens takes the post-rotary query
+    and keys, which the rotary embedding makes from them. Returns (out [D],
+    idx [k]).
+    """
+    s = lowdim_scores(project_query(q_pre, P), Kt_pre, d)
+    idx = select_topk(s, k)
+    return attend(q_post, K_post, V, idx, scale), idx
+
+
 # ---------------------------------------------------------------------------
 # Batched wrappers (loops over rows; small sizes only)
 # ---------------------------------------------------------------------------

@@ -25,7 +25,8 @@ __all__ = [
     "loki_append_keys_plane", "loki_decode_attention_plane", "loki_decode_attention_fused",
     "loki_decode_step", "loki_decode_attention_paged", "loki_append_keys_paged",
     "loki_paged_decode_workspace_size", "loki_pca_attention", "loki_pca_attention_workspace_size",
-    "loki_decode_attention_noalloc",
+    "loki_decode_attention_noalloc", "loki_decode_attention_prerotary",
+    "loki_append_keys_prerotary", "loki_decode_prerotary_workspace_size",
     "loki_project_query", "loki_score_lowdim", "loki_topk", "loki_sparse_attention",
     "loki_decode_workspace_size", "dense_decode_workspace_size",
     "loki_sparse_attention_workspace_size", "loki_calibrate_workspace_size",
@@ -515,6 +516,65 @@ def loki_pca_attention(q: torch.Tensor, Kt_lo: torch.Tensor, V_cache: torch.Tens
                                  float(scale), _dt(q), out.data_ptr(), ws.data_ptr(),
                                  _ws_bytes(ws), _stream(dev)), "loki_pca_attention")
     return out
+
+
+def loki_decode_prerotary_workspace_size(B: int, H_q: int, H_kv: int, S: int, D: int, d: int,
+                                         k: int) -> int:
+    return int(lib.loki_decode_prerotary_workspace_size(B, H_q, H_kv, S, D, d, k))
+
+
+def loki_decode_attention_prerotary(q_pre: torch.Tensor, q_post: torch.Tensor,
+                                    K_cache: torch.Tensor, V_cache: torch.Tensor,
+                                    Kt_lo: torch.Tensor, P: torch.Tensor, S: int, d: int, k: int,
+                                    scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                    selected_idx: Optional[torch.Tensor] = None,
+                                    workspace: Optional[torch.Tensor] = None
+                                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Pre-rotary variant: select on q_pre P against the plane Kt_lo of the
+    rotated pre-rotary keys, attend with q_post over the post-rotary keys
+    K_cache. Returns (out [B, H_q, D], selected_idx [B, H_q, k] int32)."""
+    dev, B, H_q, H_kv, S_max, D = _check_decode(q_pre, K_cache, V_cache, P)
+    _expect(q_post, q_pre.shape, q_pre.dtype, "q_post")
+    _cuda(q_pre, q_post)
+    _check_plane(Kt_lo, K_cache)
+    if out is None:
+        out = torch.empty_like(q_pre)
+    if selected_idx is None:
+        selected_idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+    _cuda(q_pre, out, selected_idx)
+    _expect(out, q_pre.shape, q_pre.dtype, "out")
+    _expect(selected_idx, (B, H_q, k), torch.int32, "selected_idx")
+    if S > S_max:
+        raise ValueError("S must be <= S_max")
+    ws = _ws(loki_decode_prerotary_workspace_size(B, H_q, H_kv, S, D, d, k), dev, workspace)
+    check(lib.loki_decode_attention_prerotary(
+        q_pre.data_ptr(), q_post.data_ptr(), K_cache.data_ptr(), V_cache.data_ptr(),
+        Kt_lo.data_ptr(), Kt_lo.shape[3], P.data_ptr(), B, H_q, H_kv, S, S_max, D, d, k,
+        float(scale), _dt(q_pre), out.data_ptr(), selected_idx.data_ptr(), ws.data_ptr(),
+        _ws_bytes(ws), _stream(dev)), "loki_decode_attention_prerotary")
+    return out, selected_idx
+
+
+def loki_append_keys_prerotary(K_new_pre: torch.Tensor, K_new_post: torch.Tensor,
+                               V_new: torch.Tensor, P: torch.Tensor, K_cache: torch.Tensor,
+                               V_cache: torch.Tensor, Kt_lo: torch.Tensor, pos: int) -> None:
+    """Append of the pre-rotary variant: (K_new_pre P)[:, :d_lo] to the plane,
+    K_new_post and V_new unchanged to the caches, at rows [pos, pos + T)."""
+    dev = _cuda(K_new_pre, K_new_post, V_new, P, K_cache, V_cache)
+    B, H_kv, T, D = K_new_pre.shape
+    S_max = K_cache.shape[2]
+    for t in (K_new_post, V_new):
+        _expect(t, K_new_pre.shape, K_new_pre.dtype, "K_new_post / V_new")
+    _expect(V_cache, K_cache.shape, K_new_pre.dtype, "V_cache")
+    if K_cache.dtype != K_new_pre.dtype or K_cache.shape[:2] != (B, H_kv) or K_cache.shape[3] != D:
+        raise ValueError("K_cache must be [B, H_kv, S_max, D] of the new keys' dtype")
+    if P.dtype != torch.float32 or tuple(P.shape) != (H_kv, D, D):
+        raise ValueError("P must be float32 [H_kv, D, D]")
+    _check_plane(Kt_lo, K_cache)
+    check(lib.loki_append_keys_prerotary(
+        K_new_pre.data_ptr(), K_new_post.data_ptr(), V_new.data_ptr(), P.data_ptr(),
+        K_cache.data_ptr(), V_cache.data_ptr(), Kt_lo.data_ptr(), Kt_lo.shape[3], B, H_kv, T, D,
+        S_max, pos, _dt(K_new_pre), _stream(dev)), "loki_append_keys_prerotary")
 
 
 def dense_decode_attention(q: torch.Tensor, K_cache: torch.Tensor, V_cache: torch.Tensor, S: int,

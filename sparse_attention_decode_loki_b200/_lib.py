@@ -78,6 +78,15 @@ PROTOTYPES = {
     "loki_pca_attention": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                    c_int, c_int64, c_int64, c_int, c_int, c_float, c_int,
                                    c_void_p, c_void_p, c_size_t, c_void_p]),
+    "loki_decode_prerotary_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int64, c_int, c_int,
+                                                        c_int64]),
+    "loki_decode_attention_prerotary": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                c_int, c_void_p, c_int, c_int, c_int, c_int64,
+                                                c_int64, c_int, c_int, c_int64, c_float, c_int,
+                                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "loki_append_keys_prerotary": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                           c_int64, c_int64, c_int, c_void_p]),
     "dense_decode_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int64, c_int]),
     "dense_decode_attention": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int64,
                                        c_int64, c_int, c_float, c_int, c_void_p, c_void_p, c_size_t,

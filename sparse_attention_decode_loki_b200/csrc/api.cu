@@ -731,6 +731,107 @@ loki_status loki_sparse_attention(const float* q_rot, const void* Kt_cache, cons
 
 // ---------------------------------------------------------------------------
 
+size_t loki_decode_prerotary_workspace_size(int B, int H_q, int H_kv, int64_t S, int D, int d,
+                                            int64_t k) {
+    (void)H_kv;
+    (void)d;
+    if (B < 1 || H_q < 1 || S < 1 || D < 1 || k < 1) return 0;
+    return align_up((size_t)B * H_q * D * sizeof(float)) + decode_ws(B, H_q, S, D, k).total;
+}
+
+loki_status loki_decode_attention_prerotary(const void* q_pre, const void* q_post,
+                                            const void* K_cache, const void* V_cache,
+                                            const void* Kt_lo, int d_lo, const float* P, int B,
+                                            int H_q, int H_kv, int64_t S, int64_t S_max, int D,
+                                            int d, int64_t k, float scale, loki_dtype dt,
+                                            void* out, int32_t* selected_idx, void* ws,
+                                            size_t ws_bytes, void* stream) {
+    g_last_error.clear();
+    const char* name = "loki_decode_attention_prerotary";
+    LOKI_CHECK(check_decode_common(B, H_q, H_kv, S, S_max, D, dt));
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    LOKI_REQUIRE(d >= 1 && d <= d_lo, LOKI_ERR_INVALID_ARG, "d must be in [1, d_lo] (got %d)", d);
+    LOKI_REQUIRE(k >= 1 && k <= S, LOKI_ERR_INVALID_ARG, "k must be in [1, S] (got %lld)",
+                 (long long)k);
+    LOKI_PTR(q_pre, 16);
+    LOKI_PTR(q_post, 16);
+    LOKI_PTR(K_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(Kt_lo, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(out, 16);
+    LOKI_PTR(selected_idx, 4);
+    LOKI_PTR(ws, 256);
+    const size_t qbytes = align_up((size_t)B * H_q * D * sizeof(float));
+    const DecodeWs w = decode_ws(B, H_q, S, D, k);
+    LOKI_REQUIRE(ws_bytes >= qbytes + w.total, LOKI_ERR_WORKSPACE_TOO_SMALL,
+                 "workspace %zu bytes < required %zu", ws_bytes, qbytes + w.total);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const loki::Dt t = to_dt(dt);
+    float* q_sc = at<float>(ws, 0);  // q~ = q_pre P, for the scores
+    void* dws = at<char>(ws, qbytes);
+    float* q_att = at<float>(dws, w.q_rot);  // q_post in fp32, for the attention
+    float* scores = at<float>(dws, w.scores);
+    int* done = at<int>(dws, w.done);
+    const int rows = B * H_q;
+    // the scan of the pre-rotary plane (rotating q_pre itself where it can);
+    // q_post is widened to fp32 by the identity rotation
+    if (loki::score_plane_fuses(t, H_q / H_kv, d_lo, D)) {
+        LOKI_CUDA(loki::launch_score_plane(t, q_sc, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
+                                           scores, s, false, q_pre, P),
+                  name);
+        LOKI_CUDA(loki::launch_project_query(t, q_post, nullptr, B, H_q, H_kv, D, q_att, s, done,
+                                             rows, true),
+                  name);
+    } else {
+        LOKI_CUDA(loki::launch_project_query(t, q_pre, P, B, H_q, H_kv, D, q_sc, s), name);
+        LOKI_CUDA(loki::launch_project_query(t, q_post, nullptr, B, H_q, H_kv, D, q_att, s, done,
+                                             rows),
+                  name);
+        LOKI_CUDA(loki::launch_score_plane(t, q_sc, Kt_lo, B, H_q, H_kv, S, S_max, D, d_lo, d,
+                                           scores, s, true),
+                  name);
+    }
+    return decode_tail(name, t, scores, q_att, done, dws, w, K_cache, V_cache, B, H_q, H_kv, S,
+                       S_max, D, k, scale, out, selected_idx, s);
+}
+
+loki_status loki_append_keys_prerotary(const void* K_new_pre, const void* K_new_post,
+                                       const void* V_new, const float* P, void* K_cache,
+                                       void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
+                                       int T, int D, int64_t S_max, int64_t pos, loki_dtype dt,
+                                       void* stream) {
+    g_last_error.clear();
+    LOKI_CHECK(check_dtype(dt));
+    LOKI_CHECK(check_heads(B, H_kv, H_kv, D));
+    LOKI_CHECK(check_plane(d_lo, D, dt));
+    LOKI_REQUIRE(T >= 1, LOKI_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    LOKI_REQUIRE(pos >= 0 && S_max >= 1 && pos + T <= S_max, LOKI_ERR_INVALID_ARG,
+                 "need 0 <= pos and pos + T <= S_max (pos %lld, T %d, S_max %lld)",
+                 (long long)pos, T, (long long)S_max);
+    LOKI_PTR(K_new_pre, 16);
+    LOKI_PTR(K_new_post, 16);
+    LOKI_PTR(V_new, 16);
+    LOKI_PTR(P, 16);
+    LOKI_PTR(K_cache, 16);
+    LOKI_PTR(V_cache, 16);
+    LOKI_PTR(Kt_lo, 16);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const loki::Dt t = to_dt(dt);
+    const char* name = "loki_append_keys_prerotary";
+    // the rotated pre-rotary keys go to the plane only; the post-rotary keys
+    // (identity rotation) and the values to the caches
+    LOKI_CUDA(loki::launch_rotate(t, nullptr, K_new_pre, nullptr, P, nullptr, nullptr, nullptr,
+                                  Kt_lo, d_lo, B, H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0,
+                                  false),
+              name);
+    LOKI_CUDA(loki::launch_rotate(t, nullptr, K_new_post, V_new, nullptr, nullptr, K_cache,
+                                  V_cache, nullptr, 0, B, H_kv, H_kv, T, D, S_max, pos, s, nullptr,
+                                  0, false),
+              name);
+    return LOKI_OK;
+}
+
 size_t loki_pca_attention_workspace_size(int B, int H_q, int H_kv, int64_t S, int D) {
     (void)H_kv;
     if (B < 1 || H_q < 1 || S < 1 || D < 1) return 0;

@@ -1,6 +1,9 @@
 // Rotation of rows into a KV head's PCA basis: queries, q~ = q P, and new
 // keys appended to the KV-cache, K~ = K P (the key also goes to the
-// low-dimensional key plane; its value row is copied unchanged).
+// low-dimensional key plane; its value row is copied unchanged). With no P
+// the rotation is the identity: rows are copied (queries widened to fp32,
+// keys written to the cache as they are), which the pre-rotary variant uses
+// for its post-rotary queries and keys.
 //
 // Loki (NeurIPS 2024 poster page, "Visual Insights" Figure 1 caption: keys
 // and queries are used through their PCA projection; "Loki's Computational
@@ -49,16 +52,22 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
     const int R = G + T;  // rows of the head per sequence
     const int nrows = (int)min64(kRotRows, (int64_t)B * R - r0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float* Ph = P + (int64_t)hk * D * D;
-    // the P block: 128 rows x 32 columns = 1024 float4, 4 per thread, all in flight
+    const float* Ph = P != nullptr ? P + (int64_t)hk * D * D : nullptr;
+    // the P block: 128 rows x 32 columns = 1024 float4, 4 per thread, all in
+    // flight (no P: the identity's block, so each sum is one exact product)
     float4 pv[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int it = tid + u * 256;
         const int i = it >> 3, c4 = (it & 7) * 4;
-        pv[u] = (i < D && c0 + c4 < D)
-                    ? __ldg(reinterpret_cast<const float4*>(Ph + (int64_t)i * D + c0 + c4))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int c = c0 + c4;
+        if (P == nullptr)
+            pv[u] = make_float4(i == c ? 1.f : 0.f, i == c + 1 ? 1.f : 0.f,
+                                i == c + 2 ? 1.f : 0.f, i == c + 3 ? 1.f : 0.f);
+        else
+            pv[u] = (i < D && c < D)
+                        ? __ldg(reinterpret_cast<const float4*>(Ph + (int64_t)i * D + c))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // row j of the chunk: sequence b = (r0 + j) / R, member g = (r0 + j) % R
     // (a query head for g < G, else new key g - G); 8 elements per thread and
@@ -120,9 +129,9 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
                 row = ((int64_t)page * H_kv + hk) * page_size + j % page_size;
             }
             const Tp kt = E::from_float(acc);
-            if (c < D) Kt_cache[row * D + c] = kt;
+            if (Kt_cache != nullptr && c < D) Kt_cache[row * D + c] = kt;
             if (Kt_lo != nullptr && c < d_lo) Kt_lo[row * d_lo + c] = kt;
-            if (cb == 0) {  // one column block copies the value row
+            if (V_cache != nullptr && cb == 0) {  // one column block copies the value row
                 const Tp* vs = V_new + (((int64_t)b * H_kv + hk) * T + t) * D;
                 for (int e = lane; e < D; e += 32) V_cache[row * D + e] = vs[e];
             }

@@ -118,7 +118,14 @@ def fp32_score_bound(q: np.ndarray, P: np.ndarray, Kt: np.ndarray, d: int) -> np
 
 def check_row(inp: HostInputs, b: int, h: int, gpu_idx: np.ndarray, gpu_out: np.ndarray,
               d: int, k: int, scale: float, S: Optional[int] = None,
-              gpu_scores: Optional[np.ndarray] = None) -> RowCheck:
+              gpu_scores: Optional[np.ndarray] = None,
+              attend_with: Optional[Tuple[np.ndarray, np.ndarray]] = None) -> RowCheck:
+    """One row against the oracle: the selection outside the tie band, the
+    scores (when given) within the fp32 bound, the output within OUT_TOL.
+
+    attend_with = (query [D], keys [S, D]) replaces q~ and K~ in the exact
+    attention over the selected tokens (the pre-rotary variant attends with
+    its post-rotary query and keys)."""
     wl = inp.wl
     S = wl.S if S is None else S
     hk = h // wl.G
@@ -149,7 +156,9 @@ def check_row(inp: HostInputs, b: int, h: int, gpu_idx: np.ndarray, gpu_out: np.
         f"row {(b, h)}: {len(diff)} tokens differ outside the tie band "
         f"(max |s-s_k| = {gap.max() if len(diff) else 0:.3e}, band {rel:.3e})")
     floor_only = int(np.sum(gap > rel))
-    ref = oracle.attend(q_rot, Kt, V, gi if len(diff) else I, scale)
+    qa, Ka = (q_rot, Kt) if attend_with is None else (
+        np.asarray(attend_with[0], np.float64), np.asarray(attend_with[1], np.float64)[:S])
+    ref = oracle.attend(qa, Ka, V, gi if len(diff) else I, scale)
     err = float(np.abs(gpu_out.astype(np.float64) - ref).max())
     assert err <= OUT_TOL[wl.dtype], f"row {(b, h)}: max |out - oracle| = {err:.3e}"
     return RowCheck((b, h), len(diff) == 0, len(diff), err, floor_only)

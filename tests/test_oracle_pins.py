@@ -314,3 +314,46 @@ def test_calibrate_heads_closed_form_per_head():
     for h in range(3):
         np.testing.assert_allclose(w[h], expect_w[h], rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(P[h], expect_P[h], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# the pre-rotary variant
+# ---------------------------------------------------------------------------
+
+def test_prerotary_hand_worked():
+    """Selection on the rotated pre-rotary keys (first d columns), attention
+    with the post-rotary query and keys. Worked by hand: P swaps the two
+    axes, so q~ = (2, 1) and K~pre = [[1, 0], [0.5, 0], [0, 3]]; on d = 1 the
+    scores are (2, 1, 0). Selecting on d = 2 (scores (2, 1, 3)), on the
+    unrotated keys ((0, 0, 3)) or on the post-rotary ones ((0, 2, 10)) would
+    pick token 2 instead of token 0."""
+    P = np.array([[0.0, 1.0], [1.0, 0.0]])
+    q_pre, q_post = np.array([1.0, 2.0]), np.array([1.0, 0.0])
+    K_pre = np.array([[0.0, 1.0], [0.0, 0.5], [3.0, 0.0]])
+    K_post = np.array([[0.0, 1.0], [2.0, 0.0], [5.0, 5.0]])
+    V = np.array([[10.0, 0.0], [0.0, 20.0], [7.0, 7.0]])
+    Kt_pre = oracle.rotate_keys(K_pre, P)
+    out, idx = oracle.prerotary_decode_row(q_pre, q_post, Kt_pre, K_post, V, P, 1, 1, 1.0)
+    np.testing.assert_array_equal(idx, [0])
+    np.testing.assert_array_equal(out, [10.0, 0.0])
+    # k = 2: tokens {0, 1}; post-rotary logits (0, 2)
+    out, idx = oracle.prerotary_decode_row(q_pre, q_post, Kt_pre, K_post, V, P, 1, 2, 1.0)
+    np.testing.assert_array_equal(idx, [0, 1])
+    e2 = math.exp(2.0)
+    np.testing.assert_allclose(out, [10.0 / (1 + e2), 20.0 * e2 / (1 + e2)], rtol=1e-14)
+
+
+def test_prerotary_without_rotary_is_loki():
+    """With no rotary embedding (post = pre) the variant is Loki itself: the
+    exact scores q . K_j equal q~ . K~_j because P is orthonormal."""
+    rng = np.random.default_rng(3)
+    S, D, d, k = 40, 8, 3, 7
+    K = rng.standard_normal((S, D))
+    V = rng.standard_normal((S, D))
+    q = rng.standard_normal(D)
+    P, _ = oracle.calibrate_pca(rng.standard_normal((200, D)) * np.linspace(3, 0.1, D))
+    Kt = oracle.rotate_keys(K, P)
+    out, idx = oracle.prerotary_decode_row(q, q, Kt, K, V, P, d, k, 0.4)
+    want, widx, _, _ = oracle.loki_decode_row(q, Kt, V, P, d, k, 0.4)
+    np.testing.assert_array_equal(idx, widx)
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12)

@@ -1,4 +1,6 @@
 """The seeded input generator: determinism, block independence, dtype exactness."""
+import math
+
 import numpy as np
 
 import workloads
@@ -49,3 +51,23 @@ def test_sweep_has_54_points_and_sample_rows():
     rows = workloads.sample_rows(wl, 16)
     assert len(rows) == 16 and rows[0] == (0, 0) and rows[-1] == (wl.B - 1, wl.H_q - 1)
     assert len(set(rows)) == 16
+
+
+def test_rope_is_a_position_dependent_rotation():
+    """Rotary embedding: identity at position 0, norm-preserving per column
+    pair, and q(m) . k(n) depends only on m - n."""
+    rng = np.random.default_rng(0)
+    D = 16
+    x = rng.standard_normal((5, D))
+    np.testing.assert_allclose(workloads.rope(x, np.zeros(5)), x, atol=0)
+    y = workloads.rope(x, np.arange(5) * 7.0)
+    h = D // 2
+    np.testing.assert_allclose(x[:, :h] ** 2 + x[:, h:] ** 2, y[:, :h] ** 2 + y[:, h:] ** 2,
+                               rtol=1e-12)
+    q, k = rng.standard_normal(D), rng.standard_normal(D)
+    a = workloads.rope(q[None], [9.0])[0] @ workloads.rope(k[None], [4.0])[0]
+    b = workloads.rope(q[None], [105.0])[0] @ workloads.rope(k[None], [100.0])[0]
+    assert abs(a - b) < 1e-12
+    # one hand value: D = 2, position 1, angle 1 rad
+    np.testing.assert_allclose(workloads.rope(np.array([[1.0, 0.0]]), [1.0])[0],
+                               [math.cos(1.0), math.sin(1.0)], rtol=1e-15)

@@ -216,6 +216,26 @@ def calibration_keys(wl: Workload, h_kv: int, R: Optional[np.ndarray] = None,
     return to_cache_dtype(x, wl.dtype)
 
 
+def rope(x: np.ndarray, positions: np.ndarray, base: float = 10000.0,
+         dtype: Optional[str] = None) -> np.ndarray:
+    """Rotary position embedding of rows x [..., n, D] at token positions [n].
+
+    The input-side transform that makes the post-rotary keys and queries of
+    the pre-rotary variant from the generated (pre-rotary) ones: column pair
+    (i, i + D/2) of the row at position t turns by the angle t * base^(-2i/D)
+    (the half-split pairing). Computed in fp64; rounded to `dtype` when given.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    half = D // 2
+    inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / D)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :half], x[..., half:]
+    y = np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+    return y if dtype is None else to_cache_dtype(y, dtype)
+
+
 def _threads(threads: Optional[int]) -> int:
     if threads:
         return threads
