@@ -28,10 +28,16 @@ constexpr int kTopkChunkTarget = LOKI_TOPK_CHUNK_TARGET;
 // With lens (a per-sequence length, row r belonging to sequence r / H_q) a
 // row holds lens[r / H_q] <= S keys at stride S: it selects min(k, length)
 // and pads its output with -1.
+// Rows of up to 4096 keys keep to 48 registers, so five 256-thread CTAs fit
+// on an SM: a decode's rows (640 at the Llama2-13B shape) then all start in
+// one wave on 148 SMs.
 template <int NT, int I, bool kCl>
-__global__ void __launch_bounds__(NT) k_topk(const float* __restrict__ scores, int S, int k,
-                                             int chunk, int32_t* __restrict__ out, int vec4,
-                                             const int* __restrict__ lens, int H_q) {
+constexpr int kTopkMinBlocks = (!kCl && NT * I <= 1024) ? 1280 / NT : 1;
+
+template <int NT, int I, bool kCl>
+__global__ void __launch_bounds__(NT, (kTopkMinBlocks<NT, I, kCl>)) k_topk(
+    const float* __restrict__ scores, int S, int k, int chunk, int32_t* __restrict__ out, int vec4,
+    const int* __restrict__ lens, int H_q) {
     __shared__ __align__(16) uint32_t scratch[kTkSmemWords];
     TkCluster<kCl> cl;
     cl.init();

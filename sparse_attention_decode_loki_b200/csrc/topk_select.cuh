@@ -12,7 +12,10 @@
 // shared-memory histogram (fire-and-forget atomics from registers), and one
 // block-wide scan over the bins finds the bin holding the k-th key. That also
 // gives how many keys equal to T belong to the set (ties go to the lowest
-// token indices). A compaction then writes the selected indices in ascending
+// token indices). A pass whose threshold bin is taken whole ends the search
+// early (for continuous scores the 22-bit prefix of pass 2 almost always
+// isolates the k-th key, so pass 3 rarely runs). A compaction then writes the
+// selected indices in ascending
 // token order: each warp scans its lanes' per-step counts packed as 8-bit
 // fields, and warp and CTA prefixes place every key. Every decision is an
 // integer compare, so the result is exact and deterministic.
@@ -51,15 +54,18 @@ constexpr int kTkBins2 = 2048;  // digit 2: key bits 20..10
 constexpr int kTkBins3 = 1024;  // digit 3: key bits 9..0
 constexpr int kTkMaxKeysPerThread = 32;
 
-// Shared-memory scratch of one selection: the three histograms and 64 words
-// of reduction slots.
+// Shared-memory scratch of one selection: the histograms and 64 words of
+// reduction slots. The third histogram reuses the first one's words (cleared
+// once the first pass's bin search is over), so the scratch stays small
+// enough for five 256-thread top-k CTAs per SM.
 struct TkSmem {
     uint32_t* hist1;
     uint32_t* hist2;
     uint32_t* hist3;
     int* red;
 };
-constexpr int kTkSmemWords = kTkBins1 + kTkBins2 + kTkBins3 + 64;
+constexpr int kTkSmemWords = kTkBins1 + kTkBins2 + 64;
+static_assert(kTkBins3 <= kTkBins1, "the third histogram lives in the first");
 
 // red[] slots (0..31: per-warp partial sums)
 constexpr int kRedBin = 32, kRedKrem = 33, kRedCnt = 34, kRedTotal = 35;
@@ -68,16 +74,16 @@ __device__ __forceinline__ TkSmem tk_carve(uint32_t* base) {
     TkSmem s;
     s.hist1 = base;
     s.hist2 = base + kTkBins1;
-    s.hist3 = s.hist2 + kTkBins2;
-    s.red = reinterpret_cast<int*>(s.hist3 + kTkBins3);
+    s.hist3 = base;
+    s.red = reinterpret_cast<int*>(s.hist2 + kTkBins2);
     return s;
 }
 
-// Zero the three histograms (all threads of the block; visible after the
-// next barrier).
+// Zero the histograms (all threads of the block; visible after the next
+// barrier).
 template <int NT>
 __device__ __forceinline__ void tk_zero(const TkSmem& sm) {
-    constexpr int n4 = (kTkBins1 + kTkBins2 + kTkBins3) / 4;
+    constexpr int n4 = (kTkBins1 + kTkBins2) / 4;
     for (int i = threadIdx.x; i < n4; i += NT)
         reinterpret_cast<uint4*>(sm.hist1)[i] = make_uint4(0u, 0u, 0u, 0u);
 }
@@ -227,8 +233,8 @@ __device__ __forceinline__ void tk_find_bin(const CL& cl, const uint32_t* hist, 
 //   v      this thread's I groups of keys (layout above); padding keys are 0
 //   base   global index of the CTA's first key (rank * chunk in a cluster)
 //   sm     scratch: hist1 holds this CTA's histogram of key bits 31..21 over
-//          its keys, hist2 and hist3 are zero (the call's first barrier
-//          publishes them)
+//          its keys, hist2 is zero (the call's first barrier publishes
+//          them; hist3 shares hist1's words and is cleared here)
 //   k      1 <= k <= the row's number of keys
 // Every thread of every CTA of the cluster must call it. On return every
 // thread is past its last barrier (in a cluster: past a final cluster
@@ -246,42 +252,68 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
     tk_find_bin<NT, kTkBins1, kCl, CL>(cl, sm.hist1, k, red);
     const uint32_t bin1 = (uint32_t)red[kRedBin];
     int krem = red[kRedKrem];
-    // pass 2: bits 20..10 of the keys in the threshold bin
+    // A pass whose threshold bin is taken whole ends the search: the set is
+    // then every key at or above the bin's lowest key, with no tie to break.
+    // The counts are the cluster's, so every thread takes the same branch.
+    // lo: that lowest key; T, take_T, cnt_T: the exact threshold of pass 3.
+    uint32_t lo = 0u, T = 0u;
+    int take_T = 0, cnt_T = 0;
+    bool whole = krem == red[kRedCnt];
+    if (whole) {
+        lo = bin1 << 21;
+    } else {
+        // pass 2: bits 20..10 of the keys in the threshold bin
 #pragma unroll
-    for (int i = 0; i < I; ++i) {
-        const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        for (int i = 0; i < I; ++i) {
+            const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (kk[e] != 0u && (kk[e] >> 21) == bin1) atomicAdd(&sm.hist2[(kk[e] >> 10) & 2047u], 1u);
+            for (int e = 0; e < 4; ++e)
+                if (kk[e] != 0u && (kk[e] >> 21) == bin1)
+                    atomicAdd(&sm.hist2[(kk[e] >> 10) & 2047u], 1u);
+        }
+        cl.sync();
+        // no CTA of the cluster reads the pass-1 histograms any more: clear
+        // the words pass 3 counts into (the bin search's barriers publish it)
+        for (int i = tid; i < kTkBins3 / 4; i += NT)
+            reinterpret_cast<uint4*>(sm.hist3)[i] = make_uint4(0u, 0u, 0u, 0u);
+        tk_find_bin<NT, kTkBins2, kCl, CL>(cl, sm.hist2, krem, red);
+        const uint32_t pre = (bin1 << 11) | (uint32_t)red[kRedBin];
+        krem = red[kRedKrem];
+        whole = krem == red[kRedCnt];
+        if (whole) {
+            lo = pre << 10;
+        } else {
+            // pass 3: bits 9..0 of the keys sharing the 22-bit prefix
+#pragma unroll
+            for (int i = 0; i < I; ++i) {
+                const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (kk[e] != 0u && (kk[e] >> 10) == pre) atomicAdd(&sm.hist3[kk[e] & 1023u], 1u);
+            }
+            cl.sync();
+            tk_find_bin<NT, kTkBins3, kCl, CL>(cl, sm.hist3, krem, red);
+            T = (pre << 10) | (uint32_t)red[kRedBin];
+            take_T = red[kRedKrem];  // keys equal to T in the set (the lowest-index ones)
+            cnt_T = red[kRedCnt];    // keys equal to T in the row
+        }
     }
-    cl.sync();
-    tk_find_bin<NT, kTkBins2, kCl, CL>(cl, sm.hist2, krem, red);
-    const uint32_t pre = (bin1 << 11) | (uint32_t)red[kRedBin];
-    krem = red[kRedKrem];
-    // pass 3: bits 9..0 of the keys sharing the 22-bit prefix
-#pragma unroll
-    for (int i = 0; i < I; ++i) {
-        const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if (kk[e] != 0u && (kk[e] >> 10) == pre) atomicAdd(&sm.hist3[kk[e] & 1023u], 1u);
-    }
-    cl.sync();
-    tk_find_bin<NT, kTkBins3, kCl, CL>(cl, sm.hist3, krem, red);
-    const uint32_t T = (pre << 10) | (uint32_t)red[kRedBin];
-    const int take_T = red[kRedKrem];  // keys equal to T in the set (the lowest-index ones)
-    const int cnt_T = red[kRedCnt];    // keys equal to T in the row
 
     // ---- compaction ----------------------------------------------------------
-    // per-thread masks: bit 4 i + e is element e of group i
+    // per-thread masks: bit 4 i + e is element e of group i (padding keys, 0,
+    // are never selected)
     uint32_t gtm = 0u, eqm = 0u;
 #pragma unroll
     for (int i = 0; i < I; ++i) {
         const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            gtm |= (uint32_t)(kk[e] > T) << (4 * i + e);
-            eqm |= (uint32_t)(kk[e] == T) << (4 * i + e);
+            if (whole) {
+                gtm |= (uint32_t)(kk[e] != 0u && kk[e] >= lo) << (4 * i + e);
+            } else {
+                gtm |= (uint32_t)(kk[e] > T) << (4 * i + e);
+                eqm |= (uint32_t)(kk[e] == T) << (4 * i + e);
+            }
         }
     }
     // packed per-step counts: field i (8 bits) of word i / 4; a field sums at
