@@ -131,13 +131,26 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
     const bool lane_on = sub * KV < D;
     const int G = H_q / H_kv;
     int* widx = s_idx[warp];
-    griddep_wait();  // q_rot and the selected indices come from earlier kernels
-    griddep_launch_dependents();
 
     // this warp's blocks [bcur, bend); W <= N, so no warp's range is empty
     const int64_t w = (int64_t)blockIdx.x * 8 + warp;
     int64_t bcur = w < W ? w * N / W : 0;
     const int64_t bend = w < W ? (w + 1) * N / W : 0;
+    // The first row's q~ is read before the wait: this kernel is launched
+    // behind top-k, whose CTAs let it start only after their own wait on the
+    // kernels that wrote q~ (or, without programmatic launch, after all of
+    // them). The selected indices are read after the wait.
+    float qv0[KV];
+    {
+        const float* qp = q_rot + (bcur / nblk) * D + sub * KV;
+#pragma unroll
+        for (int e = 0; e < KV; ++e)
+            qv0[e] = (lane_on && bcur < bend) ? __ldg(qp + e) * scale_log2 : 0.f;
+    }
+    bool first = true;
+    griddep_wait();  // the selected indices come from top-k
+    griddep_launch_dependents();
+
     while (bcur < bend) {
         const int64_t r = bcur / nblk;
         const int64_t rb1 = min64(bend, (r + 1) * nblk);
@@ -148,7 +161,11 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
         const int64_t unit = (int64_t)b * H_kv + h / G;
 
         float qv[KV];
-        {
+        if (first) {
+#pragma unroll
+            for (int e = 0; e < KV; ++e) qv[e] = qv0[e];
+            first = false;
+        } else {
             const float* qp = q_rot + r * D + sub * KV;
 #pragma unroll
             for (int e = 0; e < KV; ++e) qv[e] = lane_on ? __ldg(qp + e) * scale_log2 : 0.f;
@@ -251,23 +268,45 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
             // loads in flight at a time
             const float2* ml = part_ml + r + wf;
             const float* pacc = part_acc + (r + wf) * D;
-            float M = -INFINITY;
-            for (int p = lane; p < nparts; p += 32) M = fmaxf(M, __ldcg(&ml[p].x));
+            const bool col_on = 4 * lane < D;
+            // (m, l) of part p on lane p (parts past 32, rare, are re-read),
+            // and the first eight parts' columns, all in flight together
+            const float2 mlp = lane < nparts ? __ldcg(&ml[lane]) : make_float2(-INFINITY, 0.f);
+            float4 a8[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+                a8[p] = (p < nparts && col_on)
+                            ? __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            float M = mlp.x;
+            for (int p = lane + 32; p < nparts; p += 32) M = fmaxf(M, __ldcg(&ml[p].x));
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
             float Lsum = 0.f;
             float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
             if (M != -INFINITY) {
-                for (int p = lane; p < nparts; p += 32) {
-                    const float2 mlp = __ldcg(&ml[p]);
-                    Lsum += mlp.y * exp2f(mlp.x - M);
+                Lsum = lane < nparts ? mlp.y * exp2f(mlp.x - M) : 0.f;
+                for (int p = lane + 32; p < nparts; p += 32) {
+                    const float2 e = __ldcg(&ml[p]);
+                    Lsum += e.y * exp2f(e.x - M);
                 }
-#pragma unroll 8
-                for (int p = 0; p < nparts; ++p) {
-                    const float sc = exp2f(__ldcg(&ml[p].x) - M);
-                    const float4 a = 4 * lane < D ? __ldcg(reinterpret_cast<const float4*>(
-                                                        pacc + (int64_t)p * D) + lane)
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    if (p < nparts) {
+                        const float sc = exp2f(__shfl_sync(0xffffffffu, mlp.x, p) - M);
+                        A.x = fmaf(a8[p].x, sc, A.x);
+                        A.y = fmaf(a8[p].y, sc, A.y);
+                        A.z = fmaf(a8[p].z, sc, A.z);
+                        A.w = fmaf(a8[p].w, sc, A.w);
+                    }
+                }
+                for (int p = 8; p < nparts; ++p) {
+                    const float mp = p < 32 ? __shfl_sync(0xffffffffu, mlp.x, p & 31)
+                                            : __ldcg(&ml[p].x);
+                    const float sc = exp2f(mp - M);
+                    const float4 a =
+                        col_on ? __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
                     A.x = fmaf(a.x, sc, A.x);
                     A.y = fmaf(a.y, sc, A.y);
                     A.z = fmaf(a.z, sc, A.z);
