@@ -39,7 +39,6 @@ if ROOT not in sys.path:
 METRIC = "Loki decode-attn µs/layer-step, HBM GB/s (% roofline), speedup vs dense"
 UNIT = "us/layer-step"
 FALLBACK_HBM_GBS = 6650.0
-LAUNCHES_PER_DECODE = 4  # score scan, projection, top-k, sparse attention with its row merge
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB of L2
 
 
@@ -53,6 +52,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every sweep point at the Llama2-13B head shape (device-generated "
+                         "inputs, Loki decode and dense decode), one JSON line per point")
     ap.add_argument("--ncu-case", action="store_true",
                     help="run a few untimed decode, dense and append steps on seeded random "
                          "full-size buffers (a small, allocation-light program for ncu)")
@@ -344,6 +346,19 @@ def actual_bytes_per_step(workload: str):
     return sum(vals)
 
 
+def count_launches(fn) -> int:
+    """Kernels of this library that one call of fn launches (CUPTI activity
+    records through the torch profiler, taken once before any timing)."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return sum(1 for e in prof.events()
+               if e.device_type.name == "CUDA" and "loki::" in e.name)
+
+
 def run_ours(args):
     import torch
 
@@ -449,6 +464,7 @@ def run_ours(args):
     # ---- the timed region: exactly K layer-steps ------------------------------------
     decode_layer(0)
     torch.cuda.synchronize()
+    launches_per_step = count_launches(lambda: decode_layer(0))
     plan, graphs = step_graphs(decode_layer, args.steps)
     wplan, wgraphs = step_graphs(decode_layer, max(args.warmup, 1))
     with ClockSampler(local) as clk:
@@ -699,7 +715,8 @@ def run_ours(args):
                      "algorithmic_bytes": alg[dom]},
         "e2e": {"value": round(e2e_us / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_DECODE * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_per_step": launches_per_step,
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -806,6 +823,146 @@ def run_ncu_case(args):
     torch.cuda.synchronize()
 
 
+def device_inputs(wl, dev, seed: int, S_cap: int):
+    """Sweep-point inputs drawn on the device with the workload's recipe
+    (low-rank keys K = Z diag(sigma) R^T + N(0, 0.01^2) per KV head, queries
+    alike, V ~ N(0, 1)); the PCA basis and the rotated cache with its key
+    plane come from the library. Timing inputs only: parity is checked by the
+    tests on the host generator's streams."""
+    import torch
+
+    import sparse_attention_decode_loki_b200 as loki
+    import workloads
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dt = torch.bfloat16
+    D, H_kv, S = wl.D, wl.H_kv, S_cap
+    sigma = torch.exp(-torch.arange(D, dtype=torch.float32, device=dev) / wl.tau)
+    Rt = [torch.from_numpy(workloads.rotation(wl, h).T.copy()).float().to(dev) for h in range(H_kv)]
+
+    def lowrank(n, h):
+        z = torch.randn((n, D), generator=gen, device=dev) * sigma
+        return z @ Rt[h] + wl.noise_std * torch.randn((n, D), generator=gen, device=dev)
+
+    K_cal = torch.stack([lowrank(wl.n_cal, h) for h in range(H_kv)], dim=1).to(dt)
+    P, _ = loki.loki_calibrate_pca(K_cal)
+    Kt = torch.empty((wl.B, H_kv, S, D), dtype=dt, device=dev)
+    V = torch.empty_like(Kt)
+    Kt_lo = torch.empty((wl.B, H_kv, S, wl.d), dtype=dt, device=dev)
+    for b in range(wl.B):
+        Kb = torch.stack([lowrank(S, h) for h in range(H_kv)]).to(dt)[None]
+        Vb = torch.randn((1, H_kv, S, D), generator=gen, device=dev).to(dt)
+        loki.loki_append_keys(Kb, Vb, P, Kt[b:b + 1], V[b:b + 1], 0, Kt_lo=Kt_lo[b:b + 1])
+        del Kb, Vb
+    q = torch.stack([torch.stack([lowrank(1, h // wl.G)[0] for h in range(wl.H_q)])
+                     for _ in range(wl.B)]).to(dt)
+    torch.cuda.synchronize()
+    return q, Kt, V, Kt_lo, P
+
+
+def run_sweep(args):
+    """Every sweep point: Loki decode and dense decode device times (graph of
+    8 x (L2 flush, call) minus 8 x (L2 flush)), ideal-bytes HBM fraction,
+    tokens/s and the speedup over dense. S is capped where a point's cache and
+    key plane do not fit in 85 % of free device memory."""
+    import torch
+
+    import sparse_attention_decode_loki_b200 as loki
+    import workloads
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    cap = torch.cuda.Stream(dev)
+    peak, peak_kind = load_peaks()
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=sink)
+
+    def diff_us(fn, R=8, reps=3):
+        fn()
+        torch.cuda.synchronize()
+
+        def graph(body):
+            g_ = torch.cuda.CUDAGraph()
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                with torch.cuda.graph(g_, stream=cap):
+                    body()
+            stream.wait_stream(cap)
+            torch.cuda.synchronize()
+            return g_
+
+        def with_call():
+            for _ in range(R):
+                flush()
+                fn()
+
+        def flush_only():
+            for _ in range(R):
+                flush()
+
+        gw, gf = graph(with_call), graph(flush_only)
+        tw, tf = [], []
+        for i in range(reps + 1):
+            for g_, t_ in ((gw, tw), (gf, tf)):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g_.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                if i:
+                    t_.append(e0.elapsed_time(e1))
+        del gw, gf
+        return (statistics.median(tw) - statistics.median(tf)) * 1e3 / R
+
+    pts = [p for p in workloads.sweep_points()
+           if args.workload in ("llama2-13b", "sweep") or p.name.startswith(args.workload)]
+    for wl in pts:
+        free, _ = torch.cuda.mem_get_info(dev)
+        per_token = wl.elem_bytes * wl.B * wl.H_kv * (2 * wl.D + wl.d) + 4 * wl.B * wl.H_q
+        S = wl.S
+        if S * per_token > 0.85 * free:
+            S = int(0.85 * free // per_token) // 4096 * 4096
+        k = S * wl.k // wl.S
+        w2 = wl.with_(S=S, k=k)
+        q, Kt, V, Kt_lo, P = device_inputs(w2, dev, w2.seed, S)
+        B, H_q, H_kv, D, d = w2.B, w2.H_q, w2.H_kv, w2.D, w2.d
+        out = torch.empty_like(q)
+        idx = torch.empty((B, H_q, k), dtype=torch.int32, device=dev)
+        ws = torch.empty(loki.loki_decode_workspace_size(B, H_q, H_kv, S, D, d, k),
+                         dtype=torch.uint8, device=dev)
+
+        def decode():
+            loki.loki_decode_attention(q, Kt, V, P, S, d, k, w2.scale, out=out, selected_idx=idx,
+                                       workspace=ws, Kt_lo=Kt_lo)
+
+        loki_us = diff_us(decode)
+        q_rot = loki.loki_project_query(q, P).to(q.dtype)
+        dws = torch.empty(loki.dense_decode_workspace_size(B, H_q, H_kv, S, D), dtype=torch.uint8,
+                          device=dev)
+        dout = torch.empty_like(q)
+        dense_us = diff_us(lambda: loki.dense_decode_attention(q_rot, Kt, V, S, w2.scale, dout, dws))
+        ideal = w2.loki_bytes()
+        dense_bytes = w2.elem_bytes * B * H_kv * 2 * S * D
+        print(json.dumps({
+            "point": wl.name, "B": B, "S": S, "S_capped": S != wl.S, "d": d, "k": k,
+            "loki_device_us": round(loki_us, 3), "dense_device_us": round(dense_us, 3),
+            "speedup_vs_dense": round(dense_us / loki_us, 3),
+            "tokens_per_s": round(B * 1e6 / loki_us, 1),
+            "ideal_bytes": ideal, "hbm_frac_ideal_of_" + peak_kind:
+                round(ideal / (loki_us * 1e-6) / 1e9 / peak, 4),
+            "dense_hbm_frac_of_" + peak_kind:
+                round(dense_bytes / (dense_us * 1e-6) / 1e9 / peak, 4),
+            "data": "synthetic, drawn on the device"}), flush=True)
+        del q, Kt, V, Kt_lo, P, out, idx, ws, dws, dout, q_rot
+        torch.cuda.empty_cache()
+
+
 def relaunch_ranks(n: int) -> int:
     """Run this command as n ranks (one process per GPU) under torch.distributed.run."""
     import subprocess
@@ -830,6 +987,9 @@ def main():
               file=sys.stderr)
     if args.ncu_case:
         run_ncu_case(args)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -256,28 +256,33 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
         // (its own included) into out[r]: publish, count, and only the warp
         // that sees the count reach the number of parts reads the others'.
         const int nparts = (int)(wl - wf + 1);
-        __threadfence();  // each lane's partial writes are visible device-wide...
-        __syncwarp();     // ...before lane 0 counts the part as done
+        // the warp's partial writes, then lane 0 counts the part with a
+        // release-acquire add: the last part's warp sees every other part
+        __syncwarp();
         int prev = 0;
-        if (lane == 0) prev = atomicAdd(done + r, 1);
+        if (lane == 0) prev = atom_add_acq_rel_gpu(done + r, 1);
         prev = __shfl_sync(0xffffffffu, prev, 0);
+        __syncwarp();
         if (prev == nparts - 1) {
-            __threadfence();
-            // lanes share the parts: (m, l) of part p go to lane p % 32, and
-            // lane l merges columns [4 l, 4 l + 4) over all parts with eight
-            // loads in flight at a time
+            // lane l merges columns [4 l, 4 l + 4) over all parts
             const float2* ml = part_ml + r + wf;
             const float* pacc = part_acc + (r + wf) * D;
             const bool col_on = 4 * lane < D;
             // (m, l) of part p on lane p (parts past 32, rare, are re-read),
-            // and the first eight parts' columns, all in flight together
+            // and the parts' columns sixteen at a time, all sixteen loads in
+            // flight together (the first sixteen already behind the max)
+            constexpr int kPB = 16;
             const float2 mlp = lane < nparts ? __ldcg(&ml[lane]) : make_float2(-INFINITY, 0.f);
-            float4 a8[8];
+            float4 ap[kPB];
+            auto load_parts = [&](int p0) {
 #pragma unroll
-            for (int p = 0; p < 8; ++p)
-                a8[p] = (p < nparts && col_on)
-                            ? __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int j = 0; j < kPB; ++j)
+                    ap[j] = (p0 + j < nparts && col_on)
+                                ? __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)(p0 + j) * D) +
+                                         lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            };
+            load_parts(0);
             float M = mlp.x;
             for (int p = lane + 32; p < nparts; p += 32) M = fmaxf(M, __ldcg(&ml[p].x));
 #pragma unroll
@@ -290,27 +295,21 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
                     const float2 e = __ldcg(&ml[p]);
                     Lsum += e.y * exp2f(e.x - M);
                 }
+                for (int p0 = 0; p0 < nparts; p0 += kPB) {
+                    if (p0 > 0) load_parts(p0);
 #pragma unroll
-                for (int p = 0; p < 8; ++p) {
-                    if (p < nparts) {
-                        const float sc = exp2f(__shfl_sync(0xffffffffu, mlp.x, p) - M);
-                        A.x = fmaf(a8[p].x, sc, A.x);
-                        A.y = fmaf(a8[p].y, sc, A.y);
-                        A.z = fmaf(a8[p].z, sc, A.z);
-                        A.w = fmaf(a8[p].w, sc, A.w);
+                    for (int j = 0; j < kPB; ++j) {
+                        const int p = p0 + j;
+                        if (p < nparts) {
+                            const float mp = p < 32 ? __shfl_sync(0xffffffffu, mlp.x, p & 31)
+                                                    : __ldcg(&ml[p].x);
+                            const float sc = exp2f(mp - M);
+                            A.x = fmaf(ap[j].x, sc, A.x);
+                            A.y = fmaf(ap[j].y, sc, A.y);
+                            A.z = fmaf(ap[j].z, sc, A.z);
+                            A.w = fmaf(ap[j].w, sc, A.w);
+                        }
                     }
-                }
-                for (int p = 8; p < nparts; ++p) {
-                    const float mp = p < 32 ? __shfl_sync(0xffffffffu, mlp.x, p & 31)
-                                            : __ldcg(&ml[p].x);
-                    const float sc = exp2f(mp - M);
-                    const float4 a =
-                        col_on ? __ldcg(reinterpret_cast<const float4*>(pacc + (int64_t)p * D) + lane)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                    A.x = fmaf(a.x, sc, A.x);
-                    A.y = fmaf(a.y, sc, A.y);
-                    A.z = fmaf(a.z, sc, A.z);
-                    A.w = fmaf(a.w, sc, A.w);
                 }
             }
 #pragma unroll
