@@ -11,10 +11,15 @@ library itself (loki_calibrate_pca, loki_append_keys) before timing.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints ONE JSON line on rank 0. `value` is microseconds per layer-step for the
-whole job (max-over-ranks device time / (K * N)); lower is better. L2 is
-flushed (a 256 MiB write) before every timed step; flush time is excluded.
-Multi-GPU runs (torchrun) are weak-scaled replicas: the path has no exchange
-step, so ranks share nothing but the final max-reduction of their timings.
+whole job (max-over-ranks device time / (K * N)); lower is better. The K
+steps cycle through enough distinct layer caches that no step finds its
+inputs in L2; a workload too small for that flushes L2 before every step and
+the flushes are timed alone and taken out. Multi-GPU runs (torchrun) are
+weak-scaled replicas: the path has no exchange step, so ranks share nothing
+but the final max-reduction of their timings.
+
+    python bench.py --sweep        # every sweep point: Loki and dense device times
+    python bench.py --ncu-case     # a few untimed full-size calls, for ncu
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (this tier has no runnable upstream code).
