@@ -369,13 +369,15 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
     const int rows = B * H_q;
     if (K_new != nullptr) {
         // Append and decode: the first kernel rotates the queries and the new
-        // keys (writing their cache, plane and value rows); the score scan is
-        // its programmatic dependent and streams the older rows at once,
-        // waiting for it only before the tiles that hold the new rows.
+        // keys (writing their cache, plane and value rows) with at most one
+        // CTA per SM; the score scan is its programmatic dependent, runs
+        // beside it and streams every older row first, waiting for it only
+        // before the new rows.
         const int64_t pos = S - T;
         LOKI_CUDA(loki::launch_rotate(t, q, K_new, V_new, P, q_rot, const_cast<void*>(Kt_cache),
                                       const_cast<void*>(V_cache), const_cast<void*>(Kt_lo), d_lo,
-                                      B, H_q, H_kv, T, D, S_max, pos, s, done, rows, false),
+                                      B, H_q, H_kv, T, D, S_max, pos, s, done, rows, false,
+                                      nullptr, nullptr, true),
                   name);
         if (Kt_lo != nullptr) {
             const bool fuse = loki::score_plane_fuses(t, H_q / H_kv, d_lo, D);

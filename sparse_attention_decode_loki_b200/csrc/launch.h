@@ -145,7 +145,8 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
                           const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
                           int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
                           int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl,
-                          const PagedKV* pg = nullptr, const int* positions = nullptr);
+                          const PagedKV* pg = nullptr, const int* positions = nullptr,
+                          bool one_per_sm = false);
 
 // PCAAttn: softmax over the low-dimensional scores s_j = q~[:d] . K~_j[:d] of
 // all S tokens (keys from the plane Klo [B, H_kv, S_max, d_lo]), out = sum p_j

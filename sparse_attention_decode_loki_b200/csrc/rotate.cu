@@ -38,18 +38,20 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
     __shared__ float xs[kRotRows][128];
     // a programmatic dependent (the score scan) may start right away
     griddep_launch_dependents();
-    // one-dimensional grid: CTA = (row chunk, column block, KV head), head fastest
-    const int64_t bid = blockIdx.x;
     if (done != nullptr) {
         const int64_t nb = gridDim.x;
-        for (int64_t i = bid * 256 + threadIdx.x; i < n_done; i += nb * 256) done[i] = 0;
+        for (int64_t i = blockIdx.x * 256 + threadIdx.x; i < n_done; i += nb * 256) done[i] = 0;
     }
     const int ncb = (D + kRotCols - 1) / kRotCols;
+    const int R = G + T;  // rows of the head per sequence
+    // work items (row chunk, column block, KV head), head fastest, dealt to
+    // the CTAs of the grid in turn (the grid may be smaller than the items)
+    const int64_t nitems = ((int64_t)B * R + kRotRows - 1) / kRotRows * ncb * H_kv;
+    for (int64_t bid = blockIdx.x; bid < nitems; bid += gridDim.x) {
     const int hk = (int)(bid % H_kv);
     const int cb = (int)((bid / H_kv) % ncb);
     const int c0 = cb * kRotCols;
     const int64_t r0 = (bid / H_kv / ncb) * kRotRows;
-    const int R = G + T;  // rows of the head per sequence
     const int nrows = (int)min64(kRotRows, (int64_t)B * R - r0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float* Ph = P != nullptr ? P + (int64_t)hk * D * D : nullptr;
@@ -137,6 +139,8 @@ __global__ void __launch_bounds__(256) k_rotate_rows(
             }
         }
     }
+    __syncthreads();  // Ps and xs are refilled for the next item
+    }
     // hold: launched beside the score scan, this grid completes only after the
     // scan does (one waiting thread is enough), so the kernels that wait on
     // it also see the scan's scores
@@ -147,7 +151,7 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
                           const float* P, float* q_rot, void* Kt_cache, void* V_cache, void* Kt_lo,
                           int d_lo, int B, int H_q, int H_kv, int T, int D, int64_t S_max,
                           int64_t pos, cudaStream_t s, int* done, int n_done, bool pdl,
-                          const PagedKV* pg, const int* positions) {
+                          const PagedKV* pg, const int* positions, bool one_per_sm) {
     int* err = device_error_word();
     if (err == nullptr) return cudaErrorInvalidDevice;
     const int* bt = pg != nullptr ? pg->block_table : nullptr;
@@ -159,7 +163,15 @@ cudaError_t launch_rotate(Dt dt, const void* q, const void* K_new, const void* V
     const int R = G + Tn;
     if (R == 0) return cudaSuccess;
     const int64_t chunks = ((int64_t)B * R + kRotRows - 1) / kRotRows;
-    const int64_t nblocks = chunks * H_kv * ((D + kRotCols - 1) / kRotCols);
+    int64_t nblocks = chunks * H_kv * ((D + kRotCols - 1) / kRotCols);
+    if (one_per_sm) {
+        // beside the score scan: at most one CTA per SM, so the scan's CTA
+        // (9 warps at 128 registers) still fits next to it on every SM
+        DevInfo di;
+        const cudaError_t e = dev_info(&di);
+        if (e != cudaSuccess) return e;
+        nblocks = min64(nblocks, di.sm_count);
+    }
     if (nblocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
     const dim3 grid((unsigned)nblocks);
     const int hold = pdl ? 1 : 0;
@@ -182,14 +194,15 @@ cudaError_t launch_project_query(Dt dt, const void* q, const float* P, int B, in
                                  int D, float* q_rot, cudaStream_t s, int* done, int n_done,
                                  bool pdl) {
     return launch_rotate(dt, q, nullptr, nullptr, P, q_rot, nullptr, nullptr, nullptr, 0, B, H_q,
-                         H_kv, 0, D, 0, 0, s, done, n_done, pdl, nullptr, nullptr);
+                         H_kv, 0, D, 0, 0, s, done, n_done, pdl, nullptr, nullptr, pdl);
 }
 
 cudaError_t launch_append(Dt dt, const void* K_new, const void* V_new, const float* P,
                           void* Kt_cache, void* V_cache, void* Kt_lo, int d_lo, int B, int H_kv,
                           int T, int D, int64_t S_max, int64_t pos, cudaStream_t s) {
     return launch_rotate(dt, nullptr, K_new, V_new, P, nullptr, Kt_cache, V_cache, Kt_lo, d_lo, B,
-                         H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0, false, nullptr, nullptr);
+                         H_kv, H_kv, T, D, S_max, pos, s, nullptr, 0, false, nullptr, nullptr,
+                         false);
 }
 
 }  // namespace loki

@@ -18,6 +18,11 @@
 // projection runs beside it); as a step of its own it reads q~ and may be
 // launched right behind the projection (programmatic dependent launch): the
 // producer then starts streaming keys at once, and only the consumers wait.
+// In a decode step that appends its new keys first (rows [wait_row, S) of
+// every unit, written by the preceding kernel), each CTA streams its older
+// rows first and only then, after waiting for the append, gathers the new
+// rows of all its segments into tiles of their own, so the append's time
+// hides behind the stream.
 #include "common.cuh"
 #include "launch.h"
 #include "tma.cuh"
@@ -32,9 +37,6 @@ constexpr int kScoreThreads = kScoreConsumers + 32;
 #ifndef LOKI_SCORE_RING_KB
 #define LOKI_SCORE_RING_KB 96
 #endif
-#ifndef LOKI_SCORE_MINB
-#define LOKI_SCORE_MINB 1
-#endif
 constexpr int kScoreRingBytes = LOKI_SCORE_RING_KB * 1024;
 constexpr int kScoreMaxStages = 16;
 
@@ -47,8 +49,10 @@ constexpr int kScoreMaxStages = 16;
 // parts rows of column c of P that it needs in registers, prefetched one unit
 // ahead, and the per-part partial sums meet in shared memory. Without it the
 // consumers read q~ from q_rot after the preceding kernel completes.
-template <class E, int G, int NV, bool kFuseQ>
-__global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
+// kDefer: the kernel of a step that appends (wait_row < S), with the new rows
+// scanned last; without it rows at or past wait_row are not expected.
+template <class E, int G, int NV, bool kFuseQ, bool kDefer>
+__device__ __forceinline__ void score_plane_body(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
     const float* __restrict__ P, const typename E::T* __restrict__ Klo,
     float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
@@ -93,25 +97,23 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
             int i = 0;
             bool ok = true;
             // rows [wait_row, S) of every unit are written by the preceding
-            // kernel (an append): wait for it before the first tile holding one
-            bool waited = wait_row >= S;
+            // kernel (an append): the older rows of every segment stream
+            // first (phase A), then, after the wait, the new rows of all the
+            // CTA's segments are gathered into tiles of their own (phase B)
+            const bool defer = kDefer && wait_row < S;
             for (int64_t r = R0; r < R1 && ok;) {
                 const int64_t unit = r / S;
                 const int s0 = (int)(r - unit * S);
                 const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+                const int segA = defer ? max(0, min(seg, wait_row - s0)) : seg;
                 const char* src = reinterpret_cast<const char*>(Klo) + (unit * S_max + s0) * kRowBytes;
-                for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
-                    const int n = min(kTR, seg - t0);
+                for (int t0 = 0; t0 < segA; t0 += kTR, ++i) {
+                    const int n = min(kTR, segA - t0);
                     const int st = i % kStages;
                     const uint32_t ph = (uint32_t)(i / kStages) & 1u;
                     if (!mbar_wait(&empty[st], ph ^ 1u, err)) {
                         ok = false;
                         break;
-                    }
-                    if (!waited && s0 + t0 + n > wait_row) {
-                        griddep_wait();
-                        fence_proxy_async_global();  // its stores, then our bulk reads
-                        waited = true;
                     }
                     mbar_arrive_expect_tx(&full[st], (uint32_t)(n * kRowBytes));
                     bulk_load_hint(ring + (size_t)st * kTile, src + (int64_t)t0 * kRowBytes,
@@ -119,9 +121,47 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
                 }
                 r += seg;
             }
-            // a CTA that never met a new row still completes only after the
-            // preceding kernel, so the kernels after the scan see its writes
-            if (!waited) griddep_wait();
+            // the preceding kernel is complete (and, in phase B, its rows are
+            // visible to our bulk reads) before any new row is read; a CTA
+            // without new rows waits too, so the kernels after the scan also
+            // see the preceding kernel's writes
+            griddep_wait();
+            if (defer && ok) {
+                fence_proxy_async_global();  // its stores, then our bulk reads
+                int fill = 0, st = 0;
+                for (int64_t r = R0; r < R1 && ok;) {
+                    const int64_t unit = r / S;
+                    const int s0 = (int)(r - unit * S);
+                    const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+                    for (int x = max(s0, wait_row); x < s0 + seg && ok;) {
+                        if (fill == 0) {
+                            st = i % kStages;
+                            if (!mbar_wait(&empty[st], ((uint32_t)(i / kStages) & 1u) ^ 1u, err)) {
+                                ok = false;
+                                break;
+                            }
+                        }
+                        const int n = min(s0 + seg - x, kTR - fill);
+                        mbar_expect_tx(&full[st], (uint32_t)(n * kRowBytes));
+                        bulk_load_hint(ring + (size_t)st * kTile + (size_t)fill * kRowBytes,
+                                       reinterpret_cast<const char*>(Klo) +
+                                           (unit * S_max + x) * kRowBytes,
+                                       (uint32_t)(n * kRowBytes), &full[st], pol);
+                        fill += n;
+                        x += n;
+                        if (fill == kTR) {
+                            mbar_arrive(&full[st]);  // the tile's one arrival
+                            fill = 0;
+                            ++i;
+                        }
+                    }
+                    r += seg;
+                }
+                if (ok && fill > 0) {
+                    mbar_arrive(&full[st]);
+                    ++i;
+                }
+            }
             // every issued copy has landed before the CTA may exit
             for (int j = max(0, i - kStages); j < i; ++j)
                 mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, err);
@@ -156,10 +196,12 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
         if (R0 < R1) LOKI_FETCH_UNIT(R0 / S)
     bool bad = false;
     int i = 0;
+    const bool defer = kDefer && wait_row < S;  // phase A: each segment's rows below wait_row
     for (int64_t r = R0; r < R1;) {
         const int64_t unit = r / S;
         const int s0 = (int)(r - unit * S);
         const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+        const int segA = defer ? max(0, min(seg, wait_row - s0)) : seg;
         const int b = (int)(unit / H_kv), hk = (int)(unit % H_kv);
         const int64_t qrow0 = (int64_t)b * H_q + (int64_t)hk * G;
         // qv holds q~ in this thread's rotated chunk order: slot cc holds
@@ -211,8 +253,8 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
 #undef LOKI_FETCH_UNIT
 
         float* srow = scores + qrow0 * S + s0;
-        for (int t0 = 0; t0 < seg; t0 += kTR, ++i) {
-            const int n = min(kTR, seg - t0);
+        for (int t0 = 0; t0 < segA; t0 += kTR, ++i) {
+            const int n = min(kTR, segA - t0);
             const int st = i % kStages;
             const uint32_t ph = (uint32_t)(i / kStages) & 1u;
             // after a timed-out wait this warp stops consuming and stops
@@ -242,6 +284,91 @@ __global__ void __launch_bounds__(kScoreThreads, LOKI_SCORE_MINB) k_score_plane(
         }
         r += seg;
     }
+    if (!kDefer || !defer) return;
+
+    // phase B: the new rows of all the CTA's segments, packed in scan order
+    // into tiles of kTR rows; new row g of the CTA lands in slot g % kTR of
+    // its tile. Their q~ comes from q_rot, which the preceding kernel wrote.
+    griddep_wait();
+    int64_t nb_all = 0;
+    for (int64_t r = R0; r < R1;) {
+        const int64_t unit = r / S;
+        const int s0 = (int)(r - unit * S);
+        const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+        nb_all += max(0, s0 + seg - max(s0, wait_row));
+        r += seg;
+    }
+    for (int64_t g0 = 0; g0 < nb_all; g0 += kTR, ++i) {
+        const int n = (int)min64(kTR, nb_all - g0);
+        const int st = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (!bad && !mbar_wait(&full[st], ph, err)) bad = true;
+        if (!bad && tid < n) {
+            // this thread's new row: walk the CTA's segments to it
+            int64_t gi = g0 + tid, unit = 0;
+            int x = 0;
+            for (int64_t r = R0; r < R1;) {
+                unit = r / S;
+                const int s0 = (int)(r - unit * S);
+                const int seg = (int)min64(R1 - r, (int64_t)S - s0);
+                const int a0 = max(s0, wait_row), nb = max(0, s0 + seg - a0);
+                if (gi < nb) {
+                    x = a0 + (int)gi;
+                    break;
+                }
+                gi -= nb;
+                r += seg;
+            }
+            const int b = (int)(unit / H_kv), hk = (int)(unit % H_kv);
+            const int64_t qrow0 = (int64_t)b * H_q + (int64_t)hk * G;
+            const unsigned char* rowp = ring + (size_t)st * kTile + tid * kRowBytes;
+            float a[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) a[g] = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < NV; ++cc) {
+                const int c = (cc + rot) & (NV - 1);
+                const uint4 v = *reinterpret_cast<const uint4*>(rowp + c * 16);
+                float f[KV];
+                E::unpack(v, f);
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < KV; ++e) {
+                        const int col = c * KV + e;
+                        const float qc = col < d ? __ldcg(q_rot + (qrow0 + g) * D + col) : 0.f;
+                        a[g] = fmaf(qc, f[e], a[g]);
+                    }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) scores[(qrow0 + g) * S + x] = a[g];
+        }
+        __syncwarp();
+        if (lane == 0 && !bad) mbar_arrive(&empty[st]);
+    }
+}
+
+template <class E, int G, int NV, bool kFuseQ>
+__global__ void __launch_bounds__(kScoreThreads, 1) k_score_plane(
+    const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
+    const float* __restrict__ P, const typename E::T* __restrict__ Klo,
+    float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
+    int D, int d, int64_t total, int64_t per, int wait_row) {
+    score_plane_body<E, G, NV, kFuseQ, false>(q_rot, q, P, Klo, scores, err, H_q, H_kv, S, S_max,
+                                              D, d, total, per, wait_row);
+}
+
+// The kernel of a step that appends runs beside the rotation kernel, so it
+// keeps to 128 registers: 9 warps at 128 leave room on every SM for the
+// rotation's CTA (at 135 the rotation waited for the scan to end).
+template <class E, int G, int NV, bool kFuseQ>
+__global__ void __maxnreg__(128) k_score_plane_append(
+    const float* __restrict__ q_rot, const typename E::T* __restrict__ q,
+    const float* __restrict__ P, const typename E::T* __restrict__ Klo,
+    float* __restrict__ scores, int* __restrict__ err, int H_q, int H_kv, int S, int64_t S_max,
+    int D, int d, int64_t total, int64_t per, int wait_row) {
+    score_plane_body<E, G, NV, kFuseQ, true>(q_rot, q, P, Klo, scores, err, H_q, H_kv, S, S_max,
+                                             D, d, total, per, wait_row);
 }
 
 // Arguments shared by every instantiation of the launch path.
@@ -266,13 +393,14 @@ static cudaError_t plane_impl(const PlaneArgs& a, cudaStream_t s, bool pdl) {
     constexpr int kTile = kScoreConsumers * NV * 16;
     constexpr int kStages = (kScoreRingBytes / kTile) < kScoreMaxStages ? (kScoreRingBytes / kTile)
                                                                       : kScoreMaxStages;
-    auto kern = k_score_plane<E, G, NV, kFuseQ>;
+    const bool append = a.wait_row < a.S;
+    auto kern = append ? k_score_plane_append<E, G, NV, kFuseQ> : k_score_plane<E, G, NV, kFuseQ>;
     const size_t smem = (size_t)kStages * kTile;
-    static bool attr_set[64] = {};
-    if (di.device < 64 && !attr_set[di.device]) {
+    static bool attr_set[2][64] = {};
+    if (di.device < 64 && !attr_set[append][di.device]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set[di.device] = true;
+        attr_set[append][di.device] = true;
     }
     const int64_t total = (int64_t)a.B * a.H_kv * a.S;
     const int64_t resident = (int64_t)di.sm_count * occupancy((const void*)kern, kScoreThreads, smem);
