@@ -393,12 +393,12 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
         return decode_tail(name, t, scores, q_rot, done, ws, w, Kt_cache, V_cache, B, H_q, H_kv,
                            S, S_max, D, k, scale, out, selected_idx, s);
     }
-    // Many (batch, KV head) units over a low-dim key plane: one kernel does
-    // the whole step per unit, with the scores in shared memory.
-    if (Kt_lo != nullptr && loki::decode_fused_preferred(t, B, H_q, H_kv, S, D, d_lo, k)) {
-        LOKI_CUDA(loki::launch_decode_fused(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S,
-                                            S_max, d_lo, d, k, resolve_scale(scale, D), out,
-                                            selected_idx, s),
+    // Few (batch, KV head) units over a low-dim key plane: one kernel does
+    // the whole step, each unit split over a cluster of CTAs.
+    if (Kt_lo != nullptr && loki::decode_cluster_preferred(t, B, H_q, H_kv, S, D, d_lo, k)) {
+        LOKI_CUDA(loki::launch_decode_cluster(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                              S_max, d_lo, d, k, resolve_scale(scale, D), out,
+                                              selected_idx, s),
                   name);
         return LOKI_OK;
     }
@@ -619,12 +619,20 @@ loki_status loki_decode_attention_fused(const void* q, const void* Kt_cache, con
     LOKI_CHECK(check_plane(d_lo, D, dt));
     LOKI_REQUIRE(d <= d_lo, LOKI_ERR_INVALID_ARG, "d (%d) must be <= d_lo (%d)", d, d_lo);
     const loki::Dt t = to_dt(dt);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // few (batch, KV head) units: each unit split over a cluster of CTAs
+    if (loki::decode_cluster_fits(t, B, H_q, H_kv, S, D, d_lo, k)) {
+        LOKI_CUDA(loki::launch_decode_cluster(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                              S_max, d_lo, d, k, resolve_scale(scale, D), out,
+                                              selected_idx, s),
+                  "loki_decode_attention_fused");
+        return LOKI_OK;
+    }
     LOKI_REQUIRE(loki::decode_fused_fits(t, H_q, H_kv, S, D, d_lo, k), LOKI_ERR_UNSUPPORTED,
                  "the fused decode kernel takes H_q / H_kv in {1, 2, 4, 8}, S <= 8192, plane "
                  "rows of 16, 32, 64 or 128 bytes, and keys that fit in shared memory");
     LOKI_CUDA(loki::launch_decode_fused(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S, S_max,
-                                        d_lo, d, k, resolve_scale(scale, D), out, selected_idx,
-                                        static_cast<cudaStream_t>(stream)),
+                                        d_lo, d, k, resolve_scale(scale, D), out, selected_idx, s),
               "loki_decode_attention_fused");
     return LOKI_OK;
 }

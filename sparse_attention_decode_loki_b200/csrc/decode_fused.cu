@@ -381,15 +381,6 @@ bool decode_fused_fits(Dt dt, int H_q, int H_kv, int64_t S, int D, int d_lo, int
     return L.total + 1024 <= di.smem_optin;
 }
 
-bool decode_fused_preferred(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo,
-                            int64_t k) {
-    // Measured at the Llama2-13B decode shape (640 units): the split pipeline
-    // is faster, because each unit's phases run back to back inside one
-    // block, so the automatic choice does not take the fused kernel yet.
-    (void)dt, (void)B, (void)H_q, (void)H_kv, (void)S, (void)D, (void)d_lo, (void)k;
-    return false;
-}
-
 #ifndef LOKI_FUSED_U
 #define LOKI_FUSED_U 8
 #endif

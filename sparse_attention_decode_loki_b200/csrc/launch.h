@@ -68,11 +68,22 @@ cudaError_t launch_topk(const float* scores, int64_t rows, int64_t S, int64_t k,
 // top-k; plane rows of 1, 2, 4 or 8 16-byte chunks; the unit's keys and
 // selection fit in shared memory.
 bool decode_fused_fits(Dt dt, int H_q, int H_kv, int64_t S, int D, int d_lo, int64_t k);
-// Whether loki_decode_attention_plane takes the fused kernel on its own.
-bool decode_fused_preferred(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo,
-                            int64_t k);
 // The whole decode step in one kernel: rotation, score scan over the plane,
 // top-k and sparse attention, per (batch, KV head) unit; writes out and sel.
+// The same step with each (batch, KV head) unit split over a cluster of 2-8
+// CTAs (top-k through distributed shared memory), for decodes with few
+// units: fits when D = 128, G in {1, 2, 4, 8}, plane rows of 16-128 bytes,
+// S <= 8192, B * H_kv * 2 <= 2 * SMs and the keys fit in shared memory.
+bool decode_cluster_fits(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo, int64_t k);
+// Whether a plane decode takes it on its own: when it fits and there are at
+// least 16 units (measured: faster than the four-kernel pipeline from 32
+// units at S = 4096 and 40 units at S = 2048; slower for a single unit).
+bool decode_cluster_preferred(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo,
+                              int64_t k);
+cudaError_t launch_decode_cluster(Dt dt, const void* q, const float* P, const void* Klo,
+                                  const void* Kt, const void* V, int B, int H_q, int H_kv,
+                                  int64_t S, int64_t S_max, int d_lo, int d, int64_t k,
+                                  float scale, void* out, int32_t* sel, cudaStream_t s);
 cudaError_t launch_decode_fused(Dt dt, const void* q, const float* P, const void* Klo,
                                 const void* Kt, const void* V, int B, int H_q, int H_kv, int64_t S,
                                 int64_t S_max, int d_lo, int d, int64_t k, float scale, void* out,

@@ -118,7 +118,7 @@ def test_fused_repeated_calls_are_identical(loki, cuda):
 
 @pytest.mark.parametrize("over,d_lo", [
     (dict(H_q=6, H_kv=2), 32),      # G = 3
-    (dict(S=8193, k=10), 32),       # beyond the block top-k
+    (dict(S=8193, k=10), 32),       # beyond the one-CTA top-k
     (dict(S=500, k=10), 128),       # 256-byte plane rows
 ])
 def test_fused_rejects_unsupported_shapes(loki, cuda, over, d_lo):
