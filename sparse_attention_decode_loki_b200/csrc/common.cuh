@@ -71,11 +71,6 @@ __device__ __forceinline__ float group_sum_rt(float v, int w) {
     return v;
 }
 
-// Programmatic dependent launch. A kernel launched with the programmatic
-// stream-serialization attribute may start while its predecessor on the
-// stream is still running; griddep_wait() blocks until the predecessor grid
-// has completed and its writes are visible (a no-op without the attribute).
-// griddep_launch_dependents() lets the next kernel be scheduled early.
 // Atomic add with release-acquire semantics at GPU scope: the calling
 // thread's earlier writes (and those it has observed, such as its warp's
 // after a warp barrier) are visible to whoever reads the new value, and
@@ -86,6 +81,11 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
     return old;
 }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialization attribute may start while its predecessor on the
+// stream is still running; griddep_wait() blocks until the predecessor grid
+// has completed and its writes are visible (a no-op without the attribute).
+// griddep_launch_dependents() lets the next kernel be scheduled early.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" :::);
