@@ -31,8 +31,10 @@ constexpr int kTopkChunkTarget = LOKI_TOPK_CHUNK_TARGET;
 // Rows of up to 4096 keys keep to 48 registers, so five 256-thread CTAs fit
 // on an SM: a decode's rows (640 at the Llama2-13B shape) then all start in
 // one wave on 148 SMs.
+// Rows of 16384 keys (512 threads of 32 keys) keep to 64 registers, two CTAs
+// per SM.
 template <int NT, int I, bool kCl>
-constexpr int kTopkMinBlocks = (!kCl && NT * I <= 1024) ? 1280 / NT : 1;
+constexpr int kTopkMinBlocks = (!kCl && NT * I <= 1024) ? 1280 / NT : (!kCl && NT == 512) ? 2 : 1;
 
 template <int NT, int I, bool kCl>
 __global__ void __launch_bounds__(NT, (kTopkMinBlocks<NT, I, kCl>)) k_topk(
@@ -76,11 +78,15 @@ __global__ void __launch_bounds__(NT, (kTopkMinBlocks<NT, I, kCl>)) k_topk(
 #pragma unroll
     for (int i = 0; i < I; ++i) {
         const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        // only a group that reaches past the row's end holds padding (key 0)
+        const bool whole = 4 * (warp * 32 * I + 32 * i + lane) + 3 < n;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            if (kk[e] != 0u) atomicAdd(&sm.hist1[kk[e] >> 21], 1u);
+            if (whole || kk[e] != 0u) atomicAdd(&sm.hist1[kk[e] >> 21], 1u);
     }
-    tk_select<NT, I, kCl>(cl, v, base, k_row, o, sm);
+    // rows of up to 4096 keys share each SM with four or more other CTAs:
+    // searching in one warp saves the instructions of the others
+    tk_select<NT, I, kCl, 0, (!kCl && NT * I <= 1024)>(cl, v, base, k_row, o, sm);
 }
 
 // exclusive prefix sum over the block; `total` gets the block sum

@@ -42,12 +42,14 @@ namespace loki {
 namespace cg = cooperative_groups;
 
 __device__ __forceinline__ uint32_t order_key(float x) {
-    uint32_t u = __float_as_uint(x);
-    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) u = 0xff800000u;  // NaN -> -inf
-    if (u == 0x80000000u) u = 0u;                                                // -0 -> +0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    // fmaxf with -inf turns NaN into -inf (IEEE maxNum returns the operand
+    // that is a number); adding +0 turns -0 into +0
+    const uint32_t u = __float_as_uint(fmaxf(x, -INFINITY) + 0.0f);
+    // negative: all bits flipped; positive: the sign bit set
+    return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
-// (no score maps to key 0: -inf maps to 0x007fffff)
+// (no score maps to key 0: -inf maps to 0x007fffff, so every real key lies in
+// bin 3 or above of the first digit and a threshold never admits padding)
 
 constexpr int kTkBins1 = 2048;  // digit 1: key bits 31..21
 constexpr int kTkBins2 = 2048;  // digit 2: key bits 20..10
@@ -163,14 +165,81 @@ __device__ __forceinline__ int block_warp_prefix(const CL& cl, int v, int* red, 
     return lo;
 }
 
+// Given the per-bin counts of this CTA's `hist` (NB bins ordered by key,
+// 1 <= krem <= their total), warp 0 alone finds the bin holding the krem-th
+// largest counted key in two levels: lane l sums bins [l * PER, (l + 1) * PER)
+// (reading its 16-byte chunks in a lane-rotated order, so the 8 lanes of a
+// quarter-warp hit distinct banks) and a suffix scan over the lanes finds the
+// block; then lane j takes bins [j * Q, (j + 1) * Q) of that block. The bin,
+// the rank left inside it and its count go to red[] and are valid for every
+// thread on return; the caller has made hist complete (block barrier).
+template <int NB, class CL>
+__device__ __forceinline__ void tk_find_bin_warp(const CL& cl, const uint32_t* hist, int krem,
+                                                 int* red) {
+    constexpr int PER = NB / 32;  // 64 or 32
+    constexpr int NV = PER / 4;   // 16-byte chunks per lane
+    constexpr int Q = PER / 32;   // bins per lane in the second level
+    static_assert(NB % 1024 == 0 && Q >= 1, "bins");
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const uint4* h4 = reinterpret_cast<const uint4*>(hist) + lane * NV;
+        uint32_t s0 = 0u, s1 = 0u, s2 = 0u, s3 = 0u;
+        // two chunks in flight: the selecting threads still hold their keys
+#pragma unroll 2
+        for (int v = 0; v < NV; ++v) {
+            const uint4 x = h4[(v + lane) & (NV - 1)];
+            s0 += x.x;
+            s1 += x.y;
+            s2 += x.z;
+            s3 += x.w;
+        }
+        const int local = (int)(s0 + s1 + s2 + s3);
+        int tot;
+        const int above = warp_suffix_excl(local, &tot);  // keys in higher lanes' blocks
+        const uint32_t m = __ballot_sync(0xffffffffu, above < krem && above + local >= krem);
+        const int L = m ? __ffs(m) - 1 : 0;  // one lane by construction
+        const int aboveL = __shfl_sync(0xffffffffu, above, L);
+        const uint32_t* hb = hist + L * PER + lane * Q;
+        uint32_t c[Q];
+        int loc2 = 0;
+#pragma unroll
+        for (int e = 0; e < Q; ++e) {
+            c[e] = hb[e];
+            loc2 += (int)c[e];
+        }
+        int tot2;
+        const int above2 = aboveL + warp_suffix_excl(loc2, &tot2);
+        if (above2 < krem && above2 + loc2 >= krem) {
+            int cum = above2;
+            bool found = false;
+#pragma unroll
+            for (int e = Q - 1; e >= 0; --e) {
+                if (!found && cum + (int)c[e] >= krem) {
+                    red[kRedBin] = L * PER + lane * Q + e;
+                    red[kRedKrem] = krem - cum;
+                    red[kRedCnt] = (int)c[e];
+                    found = true;
+                }
+                cum += (int)c[e];
+            }
+        }
+    }
+    cl.bsync();
+}
+
 // Given per-bin counts summed over the cluster's copies of `hist` (NB bins,
 // ordered by key), find the bin holding the krem-th largest counted key.
 // Thread t owns bins [t * PER, (t + 1) * PER) and keeps their sums in
 // registers. The bin, the rank left inside it and its cluster count go to
 // red[] and are valid for every thread on return. The caller has made every
-// copy of hist complete and visible (block or cluster barrier).
-template <int NT, int NB, bool kCl, class CL>
+// copy of hist complete and visible (block or cluster barrier). With kWarp
+// (one CTA) the one-warp search above runs instead.
+template <int NT, int NB, bool kCl, class CL, bool kWarp = false>
 __device__ __forceinline__ void tk_find_bin(const CL& cl, const uint32_t* hist, int krem, int* red) {
+    if constexpr (kWarp && !kCl) {
+        tk_find_bin_warp<NB, CL>(cl, hist, krem, red);
+        return;
+    }
     constexpr int PER = NB / NT;  // 1..16
     static_assert(PER >= 1 && NB % NT == 0, "bins per thread");
     constexpr int NW = NT / 32;
@@ -239,7 +308,9 @@ __device__ __forceinline__ void tk_find_bin(const CL& cl, const uint32_t* hist, 
 // Every thread of every CTA of the cluster must call it. On return every
 // thread is past its last barrier (in a cluster: past a final cluster
 // barrier, so no CTA's shared memory is still read by another).
-template <int NT, int I, bool kCl, int kBar = 0>
+// kWarpFind: the bin searches run in one warp (fewer instructions, more
+// latency: for CTAs that share their SM with several others).
+template <int NT, int I, bool kCl, int kBar = 0, bool kWarpFind = false>
 __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT : 0)>& cl,
                                           const uint4 (&v)[I], int base, int k, int32_t* out,
                                           const TkSmem& sm) {
@@ -249,7 +320,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
     int* red = sm.red;
     // every CTA's pass-1 histogram is complete
     cl.sync();
-    tk_find_bin<NT, kTkBins1, kCl, CL>(cl, sm.hist1, k, red);
+    tk_find_bin<NT, kTkBins1, kCl, CL, kWarpFind>(cl, sm.hist1, k, red);
     const uint32_t bin1 = (uint32_t)red[kRedBin];
     int krem = red[kRedKrem];
     // A pass whose threshold bin is taken whole ends the search: the set is
@@ -268,7 +339,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
             const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                if (kk[e] != 0u && (kk[e] >> 21) == bin1)
+                if ((kk[e] >> 21) == bin1)
                     atomicAdd(&sm.hist2[(kk[e] >> 10) & 2047u], 1u);
         }
         cl.sync();
@@ -276,7 +347,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
         // the words pass 3 counts into (the bin search's barriers publish it)
         for (int i = tid; i < kTkBins3 / 4; i += NT)
             reinterpret_cast<uint4*>(sm.hist3)[i] = make_uint4(0u, 0u, 0u, 0u);
-        tk_find_bin<NT, kTkBins2, kCl, CL>(cl, sm.hist2, krem, red);
+        tk_find_bin<NT, kTkBins2, kCl, CL, kWarpFind>(cl, sm.hist2, krem, red);
         const uint32_t pre = (bin1 << 11) | (uint32_t)red[kRedBin];
         krem = red[kRedKrem];
         whole = krem == red[kRedCnt];
@@ -289,10 +360,10 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
                 const uint32_t kk[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    if (kk[e] != 0u && (kk[e] >> 10) == pre) atomicAdd(&sm.hist3[kk[e] & 1023u], 1u);
+                    if ((kk[e] >> 10) == pre) atomicAdd(&sm.hist3[kk[e] & 1023u], 1u);
             }
             cl.sync();
-            tk_find_bin<NT, kTkBins3, kCl, CL>(cl, sm.hist3, krem, red);
+            tk_find_bin<NT, kTkBins3, kCl, CL, kWarpFind>(cl, sm.hist3, krem, red);
             T = (pre << 10) | (uint32_t)red[kRedBin];
             take_T = red[kRedKrem];  // keys equal to T in the set (the lowest-index ones)
             cnt_T = red[kRedCnt];    // keys equal to T in the row
@@ -309,7 +380,7 @@ __device__ __forceinline__ void tk_select(const TkCluster<kCl, kBar, (kBar ? NT 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             if (whole) {
-                gtm |= (uint32_t)(kk[e] != 0u && kk[e] >= lo) << (4 * i + e);
+                gtm |= (uint32_t)(kk[e] >= lo) << (4 * i + e);
             } else {
                 gtm |= (uint32_t)(kk[e] > T) << (4 * i + e);
                 eqm |= (uint32_t)(kk[e] == T) << (4 * i + e);
