@@ -303,10 +303,13 @@ static loki_status check_decode_common(int B, int H_q, int H_kv, int64_t S, int6
 }
 
 // Selection and attention after the score scan (both programmatic dependents).
+// d: the columns the scores cover, q_rot's own (the attention then adds the
+// stored score and reads only the remaining key columns); 0 when the scores
+// come from other queries or keys (the pre-rotary decode).
 static loki_status decode_tail(const char* name, loki::Dt t, float* scores, float* q_rot,
                                int* done, void* ws, const DecodeWs& w, const void* Kt_cache,
                                const void* V_cache, int B, int H_q, int H_kv, int64_t S,
-                               int64_t S_max, int D, int64_t k, float scale, void* out,
+                               int64_t S_max, int D, int d, int64_t k, float scale, void* out,
                                int32_t* selected_idx, cudaStream_t s) {
     const int rows = B * H_q;
     if (loki::select_attend_fits(t, (int64_t)rows, S, D, k)) {
@@ -322,7 +325,7 @@ static loki_status decode_tail(const char* name, loki::Dt t, float* scores, floa
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_cache, V_cache, selected_idx, B, H_q, H_kv,
                                             S, S_max, D, k, resolve_scale(scale, D), out,
                                             at<float2>(ws, w.ml), at<float>(ws, w.acc), done, s,
-                                            true),
+                                            true, loki::PagedKV(), scores, d),
               name);
     return LOKI_OK;
 }
@@ -391,7 +394,7 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                       name);
         }
         return decode_tail(name, t, scores, q_rot, done, ws, w, Kt_cache, V_cache, B, H_q, H_kv,
-                           S, S_max, D, k, scale, out, selected_idx, s);
+                           S, S_max, D, d, k, scale, out, selected_idx, s);
     }
     // Few (batch, KV head) units over a low-dim key plane: one kernel does
     // the whole step, each unit split over a cluster of CTAs.
@@ -431,7 +434,7 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
                       name);
     }
     return decode_tail(name, t, scores, q_rot, done, ws, w, Kt_cache, V_cache, B, H_q, H_kv, S,
-                       S_max, D, k, scale, out, selected_idx, s);
+                       S_max, D, d, k, scale, out, selected_idx, s);
 }
 
 loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
@@ -560,7 +563,7 @@ loki_status loki_decode_attention_paged(const void* q, const void* Kt_pages, con
     LOKI_CUDA(loki::launch_sparse_attention(t, q_rot, Kt_pages, V_pages, selected_idx, B, H_q, H_kv,
                                             S_cap, S_cap, D, k, resolve_scale(scale, D), out,
                                             at<float2>(dws, w.ml), at<float>(dws, w.acc), done, s,
-                                            true, pg),
+                                            true, pg, scores, d),
               name);
     return LOKI_OK;
 }
@@ -802,8 +805,9 @@ loki_status loki_decode_attention_prerotary(const void* q_pre, const void* q_pos
                                            scores, s, true),
                   name);
     }
+    // (the scores come from the pre-rotary queries and keys: no reuse)
     return decode_tail(name, t, scores, q_att, done, dws, w, K_cache, V_cache, B, H_q, H_kv, S,
-                       S_max, D, k, scale, out, selected_idx, s);
+                       S_max, D, 0, k, scale, out, selected_idx, s);
 }
 
 loki_status loki_append_keys_prerotary(const void* K_new_pre, const void* K_new_post,

@@ -115,11 +115,15 @@ struct PagedKV {
     int64_t n_pages = 0;
     const int* lens = nullptr;
 };
+// sc_lo (optional): the decode's low-dim scores [rows, S] over the first d_sc
+// columns (q~[:d_sc] . K~[:d_sc], as the score scan wrote them); the gather
+// then reads only the remaining columns of each key row and adds the score.
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
                                     float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                                    bool pdl, const PagedKV& pg = PagedKV());
+                                    bool pdl, const PagedKV& pg = PagedKV(),
+                                    const float* sc_lo = nullptr, int d_sc = 0);
 
 // ---- paged key plane -------------------------------------------------------
 // One CTA per SM; the prefix kernel turns seq_lens into this grid's work split.

@@ -13,6 +13,10 @@
 // shuffles and, per row it touches, writes the output (a whole row) or one
 // partial; the last warp to finish a row (a per-row atomic counter) merges
 // that row's partials into the output, so no separate combine kernel runs.
+// Inside a decode the score scan has already summed each selected key's
+// products over the first d columns: given those scores (and d >= D / 2), the
+// kernel reads only columns [d, D) of the key rows and adds the stored score,
+// so the gather moves (D - d) / D of the key bytes (the value rows in full).
 #include "common.cuh"
 #include "launch.h"
 
@@ -46,32 +50,35 @@ __device__ __forceinline__ int64_t owner_warp(int64_t b, int64_t W, int64_t N) {
 // Issue the key and value loads of one batch: U rows per row group, rows
 // jb + u * GPW + grp of the staged index list (indices past n, or -1 for an
 // index outside [0, S), load nothing and give zeros; so do lanes past the
-// head dimension).
+// head dimension, and for the key, lanes whose columns the stored scores
+// cover: k_on false).
 template <int U, int GPW>
 __device__ __forceinline__ void sp_load(const int* widx, int n, int jb, int grp, const char* Kb,
-                                        const char* Vb, int64_t row_bytes, bool lane_on,
+                                        const char* Vb, int64_t row_bytes, bool lane_on, bool k_on,
                                         int (&t)[U], uint4 (&kv)[U], uint4 (&vv)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int jj = jb + u * GPW + grp;
         const int tok = jj < n ? widx[jj] : -1;
         t[u] = tok;
-        if (tok >= 0 && lane_on) {
-            kv[u] = ld_stream(Kb + (int64_t)tok * row_bytes);
-            vv[u] = ld_stream(Vb + (int64_t)tok * row_bytes);
-        } else {
-            kv[u] = make_uint4(0u, 0u, 0u, 0u);
-            vv[u] = kv[u];
+        kv[u] = make_uint4(0u, 0u, 0u, 0u);
+        vv[u] = kv[u];
+        if (tok >= 0) {
+            if (k_on) kv[u] = ld_stream(Kb + (int64_t)tok * row_bytes);
+            if (lane_on) vv[u] = ld_stream(Vb + (int64_t)tok * row_bytes);
         }
     }
 }
 
 // Fold one loaded batch into the row group's running softmax state (m, l,
-// acc) in base 2: full-D scores, then the value rows weighted by 2^(s - m).
-template <class E, int U, int LPR>
+// acc) in base 2: full-D scores (with kLo, the stored part of row jb + u *
+// GPW + grp from wsc plus the loaded columns), then the value rows weighted
+// by 2^(s - m).
+template <class E, int U, int LPR, int GPW, bool kLo>
 __device__ __forceinline__ void sp_consume(const float (&qv)[E::kVec], const int (&t)[U],
-                                           const uint4 (&kv)[U], const uint4 (&vv)[U], float& m,
-                                           float& l, float (&acc)[E::kVec]) {
+                                           const uint4 (&kv)[U], const uint4 (&vv)[U],
+                                           const float* wsc, int jb, int grp, float& m, float& l,
+                                           float (&acc)[E::kVec]) {
     constexpr int KV = E::kVec;
     float sc[U];
     float mx = m;
@@ -83,6 +90,7 @@ __device__ __forceinline__ void sp_consume(const float (&qv)[E::kVec], const int
 #pragma unroll
         for (int e = 0; e < KV; ++e) a = fmaf(qv[e], f[e], a);
         a = group_sum<LPR>(a);
+        if constexpr (kLo) a += t[u] >= 0 ? wsc[jb + u * GPW + grp] : 0.f;
         sc[u] = t[u] >= 0 ? a : -INFINITY;
         mx = fmaxf(mx, sc[u]);
     }
@@ -110,14 +118,17 @@ constexpr int kSpMinBlocks = 2;
 
 // DH: head dimension (96 or 128). The lanes keep the layout of 128 columns;
 // those past DH load nothing and write nothing.
-template <class E, int DH>
+// kLo: sc_lo [rows, S] holds each token's score over the first skip * kVec
+// columns (q~ . K~ unscaled); lanes of those columns load no key chunk.
+template <class E, int DH, bool kLo>
 __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
     const float* __restrict__ q_rot, const typename E::T* __restrict__ Kt,
     const typename E::T* __restrict__ V, const int32_t* __restrict__ idx, int H_q, int H_kv, int S,
     int64_t S_max, int k, float scale_log2, int nblk, int64_t N, int64_t W,
     float2* __restrict__ part_ml, float* __restrict__ part_acc, int* __restrict__ done,
     typename E::T* __restrict__ out, const int* __restrict__ block_table, int page_size,
-    int max_pages, int64_t n_pages, const int* __restrict__ lens, int* __restrict__ err) {
+    int max_pages, int64_t n_pages, const int* __restrict__ lens, int* __restrict__ err,
+    const float* __restrict__ sc_lo, int skip) {
     constexpr int D = DH;
     constexpr int KV = E::kVec;
     constexpr int LPR = 128 / KV;   // lanes per row
@@ -125,12 +136,15 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
     constexpr int U = kSpU;         // rows in flight per group
     constexpr int64_t kRowBytes = (int64_t)D * E::kBytes;
     __shared__ int s_idx[8][kWarpIdx];
+    __shared__ float s_sc[kLo ? 8 : 1][kLo ? kWarpIdx : 1];  // stored scores, in base 2
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int grp = lane / LPR, sub = lane % LPR;
     const bool lane_on = sub * KV < D;
+    const bool k_on = lane_on && (!kLo || sub >= skip);
     const int G = H_q / H_kv;
     int* widx = s_idx[warp];
+    float* wsc = s_sc[kLo ? warp : 0];
 
     // this warp's blocks [bcur, bend); W <= N, so no warp's range is empty
     const int64_t w = (int64_t)blockIdx.x * 8 + warp;
@@ -193,6 +207,22 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
                     const int t = lane + 32 * u;
                     tk[u] = t < n ? __ldg(ip + cb + t) : -1;
                 }
+                if constexpr (kLo) {
+                    // the scan's scores of the valid tokens (all loads in flight)
+                    const float* sp = sc_lo + r * S;
+                    float sv[kWarpIdx / 32];
+#pragma unroll
+                    for (int u = 0; u < kWarpIdx / 32; ++u) {
+                        const int t = lane + 32 * u;
+                        sv[u] = (t < n && (unsigned)tk[u] < (unsigned)S_row) ? __ldg(sp + tk[u])
+                                                                              : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kWarpIdx / 32; ++u) {
+                        const int t = lane + 32 * u;
+                        if (t < n) wsc[t] = sv[u] * scale_log2;
+                    }
+                }
 #pragma unroll
                 for (int u = 0; u < kWarpIdx / 32; ++u) {
                     const int t = lane + 32 * u;
@@ -214,8 +244,8 @@ __global__ void __launch_bounds__(256, kSpMinBlocks) k_sparse_attn(
             for (int jb = 0; jb < n; jb += GPW * U) {
                 int t[U];
                 uint4 kv[U], vv[U];
-                sp_load<U, GPW>(widx, n, jb, grp, Kb, Vb, kRowBytes, lane_on, t, kv, vv);
-                sp_consume<E, U, LPR>(qv, t, kv, vv, m, l, acc);
+                sp_load<U, GPW>(widx, n, jb, grp, Kb, Vb, kRowBytes, lane_on, k_on, t, kv, vv);
+                sp_consume<E, U, LPR, GPW, kLo>(qv, t, kv, vv, wsc, jb, grp, m, l, acc);
             }
         }
         // merge the warp's row groups (lane l and lane l + LPR hold the same columns)
@@ -332,15 +362,25 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
                                const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                int64_t S_max, int D, int64_t k, float scale, void* out,
                                float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                               bool pdl, const PagedKV& pg) {
+                               bool pdl, const PagedKV& pg, const float* sc_lo, int d_sc) {
     DevInfo di;
     cudaError_t e = dev_info(&di);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)B * H_q;
-    auto kern = k_sparse_attn<E, DH>;
+    // only whole 16-byte chunks are skipped, and the stored scores pay off
+    // once they cover half the key row (measured at D = 128, bf16: d = 64
+    // takes 4 % off the step; at d = 32 the extra score loads cost what the
+    // 64 bytes fewer per key row save, the random gather being bound by its
+    // row count more than its bytes)
+    const int skip = (sc_lo != nullptr && d_sc < D && d_sc % E::kVec == 0 && 2 * d_sc >= D)
+                         ? d_sc / E::kVec
+                         : 0;
+    auto kern = skip > 0 ? k_sparse_attn<E, DH, true> : k_sparse_attn<E, DH, false>;
     // the gathers in flight live in L1: the smallest shared split that still
-    // holds two CTAs' staged indices (8 KB each, plus 1 KB reserved per CTA)
-    const int pct = (2 * (8 + 1) * 1024 * 100 + di.smem_optin - 1) / di.smem_optin + 1;
+    // holds two CTAs' staged indices (8 KB each, 16 KB with the stored
+    // scores, plus 1 KB reserved per CTA)
+    const int kb = skip > 0 ? 16 : 8;
+    const int pct = (2 * (kb + 1) * 1024 * 100 + di.smem_optin - 1) / di.smem_optin + 1;
     e = prefer_carveout((const void*)kern, pct);
     if (e != cudaSuccess) return e;
     const int64_t nblk = (k + kBlk - 1) / kBlk;
@@ -359,25 +399,29 @@ static cudaError_t sparse_impl(const float* q_rot, const void* Kt, const void* V
                          static_cast<const T*>(Kt), static_cast<const T*>(V), idx, H_q, H_kv,
                          (int)S, S_max, (int)k, scale * kLog2e, (int)nblk, N, W, part_ml,
                          part_acc, done, static_cast<T*>(out), pg.block_table, pg.page_size,
-                         pg.max_pages, pg.n_pages, pg.lens, device_error_word());
+                         pg.max_pages, pg.n_pages, pg.lens, device_error_word(),
+                         skip > 0 ? sc_lo : nullptr, skip);
 }
 
 cudaError_t launch_sparse_attention(Dt dt, const float* q_rot, const void* Kt, const void* V,
                                     const int32_t* idx, int B, int H_q, int H_kv, int64_t S,
                                     int64_t S_max, int D, int64_t k, float scale, void* out,
                                     float2* part_ml, float* part_acc, int* done, cudaStream_t s,
-                                    bool pdl, const PagedKV& pg) {
+                                    bool pdl, const PagedKV& pg, const float* sc_lo, int d_sc) {
     if (D != 96 && D != 128) return cudaErrorInvalidValue;
     if (dt == kF32)
         return D == 96 ? sparse_impl<ElemF32, 96>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
-                                                  scale, out, part_ml, part_acc, done, s, pdl, pg)
+                                                  scale, out, part_ml, part_acc, done, s, pdl, pg,
+                                                  sc_lo, d_sc)
                        : sparse_impl<ElemF32, 128>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D,
                                                    k, scale, out, part_ml, part_acc, done, s, pdl,
-                                                   pg);
+                                                   pg, sc_lo, d_sc);
     return D == 96 ? sparse_impl<ElemBF16, 96>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
-                                               scale, out, part_ml, part_acc, done, s, pdl, pg)
+                                               scale, out, part_ml, part_acc, done, s, pdl, pg,
+                                               sc_lo, d_sc)
                    : sparse_impl<ElemBF16, 128>(q_rot, Kt, V, idx, B, H_q, H_kv, S, S_max, D, k,
-                                                scale, out, part_ml, part_acc, done, s, pdl, pg);
+                                                scale, out, part_ml, part_acc, done, s, pdl, pg,
+                                                sc_lo, d_sc);
 }
 
 }  // namespace loki

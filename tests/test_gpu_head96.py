@@ -42,6 +42,7 @@ DECODE_CASES = [
     ("split-long", dict(B=1, H_q=4, H_kv=4, S=9000, d=24, k=2500), 9000, 32),
     ("f32-rows", dict(B=2, H_q=4, H_kv=2, S=700, d=20, k=90, dtype="f32"), 720, None),
     ("small-k", dict(B=3, H_q=2, H_kv=2, S=64, d=8, k=5), 64, 16),
+    ("stored-scores-d48", dict(B=2, H_q=4, H_kv=4, S=3000, d=48, k=1200), 3000, 48),
 ]
 
 

@@ -74,6 +74,7 @@ CASES = [
     ("full-and-partial-p256", dict(B=3, H_q=2, H_kv=2, d=32), [4096, 300, 2049], 256, 16, 512, 32),
     ("gqa4-p128", dict(B=3, H_q=16, H_kv=4, d=16), [1500, 4000, 129], 128, 32, 300, 16),
     ("f32-p32", dict(B=3, H_q=2, H_kv=2, d=20, dtype="f32"), [700, 5, 333], 32, 24, 90, 32),
+    ("stored-scores-d64", dict(B=3, H_q=4, H_kv=4, d=64), [3000, 1200, 77], 32, 100, 600, 64),
 ]
 
 
