@@ -184,7 +184,9 @@ LOKI_API loki_status loki_decode_attention_plane(const void* q, const void* Kt_c
  *   results, same workspace size (loki_decode_workspace_size with S).
  * The query rotation and the key rotation run in one kernel; the score scan
  * starts streaming rows [0, pos) at once and waits for that kernel only
- * before reading the new rows.
+ * before reading the new rows. With a key plane and few (batch, KV head)
+ * units (where loki_decode_attention_plane runs as one kernel) the step runs
+ * the append's rotation and then that single decode kernel behind it.
  *   requires 1 <= T, 0 <= pos, pos + T <= S_max, 1 <= k <= pos + T
  */
 LOKI_API loki_status loki_decode_step(const void* q, const void* K_new, const void* V_new,

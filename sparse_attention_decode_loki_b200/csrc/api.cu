@@ -370,6 +370,20 @@ static loki_status decode_impl(const char* name, const void* q, const void* Kt_c
     float* scores = at<float>(ws, w.scores);
     int* done = at<int>(ws, w.done);
     const int rows = B * H_q;
+    if (K_new != nullptr && Kt_lo != nullptr &&
+        loki::decode_cluster_preferred(t, B, H_q, H_kv, S, D, d_lo, k)) {
+        // Few units: the append's rotation, then the one-kernel cluster decode
+        // (which rotates its own queries) as its programmatic dependent
+        LOKI_CUDA(loki::launch_append(t, K_new, V_new, P, const_cast<void*>(Kt_cache),
+                                      const_cast<void*>(V_cache), const_cast<void*>(Kt_lo), d_lo,
+                                      B, H_kv, T, D, S_max, S - T, s),
+                  name);
+        LOKI_CUDA(loki::launch_decode_cluster(t, q, P, Kt_lo, Kt_cache, V_cache, B, H_q, H_kv, S,
+                                              S_max, d_lo, d, k, resolve_scale(scale, D), out,
+                                              selected_idx, s, true),
+                  name);
+        return LOKI_OK;
+    }
     if (K_new != nullptr) {
         // Append and decode: the first kernel rotates the queries and the new
         // keys (writing their cache, plane and value rows) with at most one

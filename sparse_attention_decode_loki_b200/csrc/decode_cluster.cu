@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(kCdThreads, 2) k_decode_cluster(
     }
     __syncthreads();
     griddep_wait();  // inputs may come from the preceding kernel (an append)
+    fence_proxy_async_global();  // whose stores precede our bulk reads
 
     // ---- 0. start the key stream; rotate the queries meanwhile ------------------
     const uint64_t pol = l2_policy_evict_first();
@@ -457,6 +458,7 @@ static int cluster_size_for(int64_t units, int sm_count) {
 
 struct ClusterShape {
     int cl, chunk, gi;
+    bool pdl = false;  // launched as a programmatic dependent (behind an append)
 };
 
 static bool cluster_shape(Dt dt, int B, int H_q, int H_kv, int64_t S, int D, int d_lo, int64_t k,
@@ -515,13 +517,15 @@ static cudaError_t cluster_impl(const ClusterShape& sh, const void* q, const flo
     cfg.blockDim = dim3(kCdThreads);
     cfg.dynamicSmemBytes = (size_t)L.total;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)sh.cl;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = sh.pdl ? 2 : 1;
     using T = typename E::T;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), P, static_cast<const T*>(Klo),
                               static_cast<const T*>(Kt), static_cast<const T*>(V), H_q, H_kv, G,
@@ -564,11 +568,12 @@ static cudaError_t cluster_nv(int nv, const ClusterShape& sh, const void* q, con
 cudaError_t launch_decode_cluster(Dt dt, const void* q, const float* P, const void* Klo,
                                   const void* Kt, const void* V, int B, int H_q, int H_kv,
                                   int64_t S, int64_t S_max, int d_lo, int d, int64_t k,
-                                  float scale, void* out, int32_t* sel, cudaStream_t s) {
+                                  float scale, void* out, int32_t* sel, cudaStream_t s, bool pdl) {
     int* err = device_error_word();
     if (err == nullptr) return cudaErrorInvalidDevice;
     ClusterShape sh;
     if (!cluster_shape(dt, B, H_q, H_kv, S, 128, d_lo, k, &sh)) return cudaErrorInvalidValue;
+    sh.pdl = pdl;
     const int nv = d_lo * (dt == kF32 ? 4 : 2) / 16;
     if (dt == kF32)
         return cluster_nv<ElemF32>(nv, sh, q, P, Klo, Kt, V, B, H_q, H_kv, S, S_max, d, k, scale,

@@ -83,7 +83,8 @@ bool decode_cluster_preferred(Dt dt, int B, int H_q, int H_kv, int64_t S, int D,
 cudaError_t launch_decode_cluster(Dt dt, const void* q, const float* P, const void* Klo,
                                   const void* Kt, const void* V, int B, int H_q, int H_kv,
                                   int64_t S, int64_t S_max, int d_lo, int d, int64_t k,
-                                  float scale, void* out, int32_t* sel, cudaStream_t s);
+                                  float scale, void* out, int32_t* sel, cudaStream_t s,
+                                  bool pdl = false);
 cudaError_t launch_decode_fused(Dt dt, const void* q, const float* P, const void* Klo,
                                 const void* Kt, const void* V, int B, int H_q, int H_kv, int64_t S,
                                 int64_t S_max, int d_lo, int d, int64_t k, float scale, void* out,

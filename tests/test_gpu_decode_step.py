@@ -45,6 +45,8 @@ CASES = [
     ("split-rows-T4", dict(B=4, H_q=8, H_kv=8, S=3000, k=400), 4, 3100, None),
     ("gqa4-plane-T3", dict(B=2, H_q=16, H_kv=4, S=2049, d=16, k=300), 3, 2100, 16),
     ("f32-plane", dict(B=2, H_q=4, H_kv=2, S=700, k=90, dtype="f32"), 2, 720, 32),
+    # 32 units: the append, then the one-kernel cluster decode behind it
+    ("cluster-plane-T4", dict(B=2, H_q=32, H_kv=16, S=2500, k=300), 4, 2600, 32),
 ]
 
 
@@ -92,11 +94,21 @@ def test_decode_step_exact_basis_matches_oracle(loki, cuda, name, over, T, S_max
     assert parity.summarize(checks)["rows"] == wl.B * wl.H_q
 
 
-@pytest.mark.parametrize("plane", [False, True])
-def test_decode_step_equals_append_then_decode(loki, cuda, plane):
+SEPARATE = [
+    # base workload, overrides, plane: 160 units (the staged kernels) and the
+    # Llama2-7B shape, 32 units (append, then the cluster decode)
+    ("llama2-13b", dict(B=4, S=4096), False),
+    ("llama2-13b", dict(B=4, S=4096), True),
+    ("llama2-7b", dict(B=1, S=4096), True),
+]
+
+
+@pytest.mark.parametrize("base,over,plane", SEPARATE,
+                         ids=["13b-rows", "13b-plane", "7b-plane-cluster"])
+def test_decode_step_equals_append_then_decode(loki, cuda, base, over, plane):
     import torch
-    wl = workloads.get("llama2-13b").with_(B=4, S=4096, name="step-vs-separate")
-    inp = parity.host_inputs(wl.with_(B=4))
+    wl = workloads.get(base).with_(name=f"step-vs-separate-{base}", **over)
+    inp = parity.host_inputs(wl)
     T, S_max = 1, 4100
     pos = wl.S - T
     dt = parity.torch_dtype(wl)
