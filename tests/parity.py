@@ -6,7 +6,7 @@ so both paths consume identical bytes and nothing fed to the oracle comes
 from the CUDA path. The GPU result is then compared with the oracle on the
 same bytes.
 
-Tolerances (from the spec contract of this library):
+Tolerances (the accuracy contract of this library):
   * selected index sets are bit-exact, except for tokens whose low-dimensional
     score lies within 1e-3 relative of the k-th score. The CUDA path computes
     q~ and the scores in fp32 (as the contract asks), and an fp32 sum cannot
