@@ -702,6 +702,7 @@ def run_ours(args):
             actual / (us_per_step_rank * 1e-6) / 1e9 / peak, 4)),
         "actual_bytes_per_step": actual,
         "ideal_bytes_per_step": step_bytes,
+        "moved_bytes_per_step": wl.moved_bytes(),
         "single_layer_graph_us": round(statistics.mean(single), 3),
         "decode_device_us": round(decode_device_us, 3),
         "fused_kernel_device_us": None if fused_us is None else round(fused_us, 3),
@@ -961,6 +962,8 @@ def run_sweep(args):
             "tokens_per_s": round(B * 1e6 / loki_us, 1),
             "ideal_bytes": ideal, "hbm_frac_ideal_of_" + peak_kind:
                 round(ideal / (loki_us * 1e-6) / 1e9 / peak, 4),
+            "moved_bytes": w2.moved_bytes(), "hbm_frac_moved_of_" + peak_kind:
+                round(w2.moved_bytes() / (loki_us * 1e-6) / 1e9 / peak, 4),
             "dense_hbm_frac_of_" + peak_kind:
                 round(dense_bytes / (dense_us * 1e-6) / 1e9 / peak, 4),
             "data": "synthetic, drawn on the device"}), flush=True)

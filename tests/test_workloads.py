@@ -71,3 +71,16 @@ def test_rope_is_a_position_dependent_rotation():
     # one hand value: D = 2, position 1, angle 1 rad
     np.testing.assert_allclose(workloads.rope(np.array([[1.0, 0.0]]), [1.0])[0],
                                [math.cos(1.0), math.sin(1.0)], rtol=1e-15)
+
+
+def test_moved_bytes_drop_only_the_reused_key_columns():
+    """With d >= D / 2 (whole 16-byte chunks) the gather skips key columns
+    [0, d); otherwise a step moves the ideal bytes."""
+    wl = workloads.get("llama2-13b")
+    assert wl.moved_bytes() == wl.loki_bytes()  # d = 32 < D / 2
+    pt = [p for p in workloads.sweep_points() if p.d == 64][0]
+    assert pt.moved_bytes() == pt.loki_bytes() - 2 * pt.B * pt.H_q * pt.k * 64
+    odd = pt.with_(d=68)  # 68 bf16 columns are not whole 16-byte chunks
+    assert odd.moved_bytes() == odd.loki_bytes()
+    f32 = pt.with_(dtype="f32", d=64)
+    assert f32.moved_bytes() == f32.loki_bytes() - 4 * f32.B * f32.H_q * f32.k * 64

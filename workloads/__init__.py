@@ -84,6 +84,16 @@ class Workload:
         e = self.elem_bytes
         return e * (self.B * self.H_kv * self.S * self.d + self.B * self.H_q * 2 * self.k * self.D)
 
+    def moved_bytes(self) -> int:
+        """loki_bytes less the key columns the attention does not re-read:
+        with d >= D / 2 (d a whole number of 16-byte chunks, d < D) it adds
+        the scan's stored score of each selected token and reads only key
+        columns [d, D)."""
+        e = self.elem_bytes
+        chunk = 16 // e
+        reuse = 2 * self.d >= self.D and self.d % chunk == 0 and self.d < self.D
+        return self.loki_bytes() - (e * self.B * self.H_q * self.k * self.d if reuse else 0)
+
     def dense_bytes(self) -> int:
         e = self.elem_bytes
         return e * self.B * self.H_kv * 2 * self.S * self.D
