@@ -9,13 +9,13 @@
 // most-significant-digit radix select finds the k-th largest key T in three
 // passes over the digits 31..21, 20..10 and 9..0 (2048, 2048 and 1024 bins):
 // each pass adds every key that still matches the known prefix into a
-// shared-memory histogram (fire-and-forget atomics from registers), and one
-// block-wide scan over the bins finds the bin holding the k-th key. That also
-// gives how many keys equal to T belong to the set (ties go to the lowest
-// token indices). A pass whose threshold bin is taken whole ends the search
-// early (for continuous scores the 22-bit prefix of pass 2 almost always
-// isolates the k-th key, so pass 3 rarely runs). A compaction then writes the
-// selected indices in ascending
+// shared-memory histogram (fire-and-forget atomics from registers), and a
+// scan over the bins (block-wide, or in one warp when several CTAs share the
+// SM) finds the bin holding the k-th key. That also gives how many keys equal
+// to T belong to the set (ties go to the lowest token indices). A pass whose
+// threshold bin is taken whole ends the search early (for continuous scores
+// the 22-bit prefix of pass 2 almost always isolates the k-th key, so pass 3
+// rarely runs). A compaction then writes the selected indices in ascending
 // token order: each warp scans its lanes' per-step counts packed as 8-bit
 // fields, and warp and CTA prefixes place every key. Every decision is an
 // integer compare, so the result is exact and deterministic.
