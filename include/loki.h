@@ -147,7 +147,11 @@ LOKI_API size_t loki_decode_workspace_size(int B, int H_q, int H_kv, int64_t S, 
  *   out     [B, H_q, D] (dt): softmax over the k selected tokens only
  *   selected_idx [B, H_q, k] int32: the k tokens with the largest
  *           low-dimensional score, ties to the lower index, ascending
- * Arithmetic: fp32 (q~, scores, softmax, accumulation) on dt inputs.
+ * Arithmetic: fp32 (q~, scores, softmax, accumulation) on dt inputs. When
+ * d >= D / 2 (and d * sizeof(dt) is a multiple of 16 bytes), each selected
+ * token's full-D score is its low-dimensional score (already computed for
+ * the selection) plus the product over columns [d, D), so the gather reads
+ * only those columns of its key row.
  */
 LOKI_API loki_status loki_decode_attention(const void* q, const void* Kt_cache, const void* V_cache,
                                   const float* P, int B, int H_q, int H_kv, int64_t S,
